@@ -1,0 +1,520 @@
+"""Benchmark of the NVFP4 MoE expert layer on B200.
+
+A step is one forward pass of the expert layer over one batch of synthetic
+tokens, through the library's C ABI: routing + dispatch with fused NVFP4
+quantization (moe_route_permute), the expert FFN on the tcgen05 tensor cores
+(moe_expert_fwd: grouped GEMM1 + SwiGLU + amax, requantization, grouped
+GEMM2) and the weighted combine (moe_combine). Inputs are resident in HBM when
+the timed region starts; the weights (6.8 GB of NVFP4 at the full size) are
+quantized once before timing, as they would be once per weight update.
+
+The metric is the expert-FFN forward throughput, 6 * T * k * d * f useful
+FLOPs per step (unpadded routed rows), in TFLOPS. The same run also measures
+the companion kernels: the quantizers (GB/s against HBM bandwidth) and the
+MXFP8 backward GEMMs (TFLOPS against the FP8 peak).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                [--workload full_moe|small_moe] [--router uniform|zipf]
+For N > 1 launch under torchrun: every rank runs an independent replica of the
+workload on its own GPU (the path has no exchange step on one node; see the
+design notes), timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 expert-FFN fwd TFLOPS (% of B200 FP4 peak); quantizer HBM GB/s"
+# dram__bytes_read.sum + dram__bytes_write.sum of moe_expert_fwd's kernels per
+# call, from the ncu capture summarised in profiles/; None until captured for
+# the current kernels.
+EXPERT_FWD_DRAM_BYTES = None
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_burst": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_burst": 1590.0, "bf16_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        self.proc = None
+        self.lines = []
+        try:
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        loaded = [m for m in mhz if mx and m > 0.3 * mx] or mhz
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# workload setup (device)
+# ---------------------------------------------------------------------------
+def setup_layer(M, synth, torch, dev, shape, router, seed_base=0):
+    T, d, f, E, k = shape.T, shape.d, shape.f, shape.E, shape.k
+    logits_np = (synth.logits_uniform_np(seed_base + 2, T, E) if router == "uniform"
+                 else synth.logits_zipf_np(seed_base + 2, T, E))
+    L = {"T": T, "d": d, "f": f, "E": E, "k": k}
+    L["logits_host"] = torch.from_numpy(logits_np).pin_memory()
+    L["logits"] = L["logits_host"].to(dev)
+    L["x"] = synth.rows_torch(seed_base, synth.TAG_X, 0, T, d, 1.0, dev)
+    L["x_host"] = L["x"].cpu().pin_memory()
+    R = M.max_rows(T, k, E)
+    L["R"] = R
+    L["idx"] = torch.empty(T, k, dtype=torch.int32, device=dev)
+    L["w"] = torch.empty(T, k, device=dev)
+    L["off"] = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    L["pos"] = torch.empty(T, k, dtype=torch.int32, device=dev)
+    L["tok"] = torch.empty(R, dtype=torch.int32, device=dev)
+    L["xq"] = torch.empty(R, d // 2, dtype=torch.uint8, device=dev)
+    L["xq_sc"] = torch.empty(R * d // 16, dtype=torch.uint8, device=dev)
+    L["x_ts"] = torch.empty(1, device=dev)
+    L["ws"] = torch.empty(M.moe_route_permute_workspace_size(T, E, k), dtype=torch.uint8,
+                          device=dev)
+
+    def qweights(tag, rows, cols):
+        c = torch.empty(E * rows, cols // 2, dtype=torch.uint8, device=dev)
+        s = torch.empty(E * rows * cols // 16, dtype=torch.uint8, device=dev)
+        t = torch.empty(E, device=dev)
+        for e in range(E):
+            wb = synth.expert_weight_torch(seed_base + 1, tag, e, rows, cols, dev)
+            M.nvfp4_quantize(wb, c[e * rows:(e + 1) * rows],
+                             s[e * rows * cols // 16:(e + 1) * rows * cols // 16], t[e:e + 1],
+                             layout=M.LAYOUT_MMA)
+            del wb
+        return c, s, t
+
+    L["w1"] = qweights(synth.TAG_W1, 2 * f, d)
+    L["w2"] = qweights(synth.TAG_W2, d, f)
+    L["h"] = torch.empty(R, f, dtype=torch.bfloat16, device=dev)
+    L["hq"] = torch.empty(R, f // 2, dtype=torch.uint8, device=dev)
+    L["hq_sc"] = torch.empty(R * f // 16, dtype=torch.uint8, device=dev)
+    L["h_amax"] = torch.empty(E, device=dev)
+    L["h_ts"] = torch.empty(E, device=dev)
+    L["y"] = torch.empty(R, d, dtype=torch.bfloat16, device=dev)
+    L["out"] = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    L["out_host"] = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    return L
+
+
+KERNELS_PER_STEP = {"moe_route_permute": 7, "moe_expert_fwd": 3, "moe_combine": 1}
+
+
+def layer_calls(M, L):
+    def route():
+        M.moe_route_permute(L["logits"], L["x"], L["k"], 1, L["idx"], L["w"], L["off"], L["pos"],
+                            L["tok"], L["xq"], L["xq_sc"], L["x_ts"], L["ws"])
+
+    def experts():
+        M.moe_expert_fwd(L["xq"], L["xq_sc"], L["x_ts"], L["off"], L["E"], L["d"], L["f"],
+                         *L["w1"], *L["w2"], L["h"], L["hq"], L["hq_sc"], L["h_amax"], L["h_ts"],
+                         L["y"], L["R"])
+
+    def combine():
+        M.moe_combine(L["y"], L["pos"], L["w"], L["out"])
+
+    return [("moe_route_permute", route), ("moe_expert_fwd", experts), ("moe_combine", combine)]
+
+
+def time_calls(torch, calls, steps):
+    """Run `steps` steps of the calls back to back on the current stream with a
+    CUDA event between calls; returns (total ms, {call: mean ms})."""
+    n = len(calls)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for s in range(steps):
+        ev[s][0].record()
+        for i, (_, fn) in enumerate(calls):
+            fn()
+            ev[s][i + 1].record()
+    end.record()
+    torch.cuda.synchronize()
+    per = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps
+           for i, (name, _) in enumerate(calls)}
+    return start.elapsed_time(end), per
+
+
+def time_kernel(torch, fn, reps, flush):
+    """Median device time of fn over reps runs, flushing L2 before each run."""
+    times = []
+    for _ in range(reps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+# ---------------------------------------------------------------------------
+# companion measurements: quantizers and the MXFP8 backward GEMMs
+# ---------------------------------------------------------------------------
+def companions(M, synth, torch, dev, L, peaks, reps=10):
+    res = {}
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    hbm = peaks["hbm_gbs"]
+    T, d, f, E, k = L["T"], L["d"], L["f"], L["E"], L["k"]
+
+    def gbs(name, fn, elems, bytes_per_elem):
+        ms = time_kernel(torch, fn, reps, flush)
+        g = elems * bytes_per_elem / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "GB/s": round(g, 1), "frac_hbm": round(g / hbm, 3),
+                     "elements": elems, "algorithmic_bytes_per_elem": bytes_per_elem}
+
+    # NVFP4 quantization of the layer input x, one pass (amax given) and two passes
+    codes = torch.empty(T, d // 2, dtype=torch.uint8, device=dev)
+    sc = torch.empty(T * d // 16, dtype=torch.uint8, device=dev)
+    ts = torch.empty(1, device=dev)
+    am = torch.empty(1, device=dev)
+    M.nvfp4moe_amax_bf16(L["x"], am)
+    gbs("nvfp4_quantize_1pass", lambda: M.nvfp4_quantize(L["x"], codes, sc, ts, amax_in=am,
+                                                         layout=M.LAYOUT_MMA), T * d, 2.5625)
+    gbs("nvfp4_quantize_2pass", lambda: M.nvfp4_quantize(L["x"], codes, sc, ts,
+                                                         layout=M.LAYOUT_MMA), T * d, 2.5625)
+    del codes, sc
+    # combine payload: RHT32 + NVFP4 / MXFP8 of the routed rows [T*k x d]
+    Rr = T * k
+    chans = synth.outlier_channels(5, d, 16)
+    pay = synth.payload_rows_torch(5, 0, Rr, d, chans, dev)
+    pc4 = torch.empty(Rr, d // 2, dtype=torch.uint8, device=dev)
+    ps4 = torch.empty(Rr, d // 16, dtype=torch.uint8, device=dev)
+    pts = torch.empty(1, device=dev)
+    pam = torch.empty(1, device=dev).fill_(1000.0)
+    gbs("rht32_nvfp4_1pass", lambda: M.rht32_quantize(pay, 11, M.FMT_NVFP4, pc4, ps4, pts,
+                                                      amax_in=pam), Rr * d, 2.5625)
+    gbs("rht32_nvfp4_2pass", lambda: M.rht32_quantize(pay, 11, M.FMT_NVFP4, pc4, ps4, pts),
+        Rr * d, 2.5625)
+    del pc4, ps4
+    pc8 = torch.empty(Rr, d, dtype=torch.uint8, device=dev)
+    ps8 = torch.empty(Rr, d // 32, dtype=torch.uint8, device=dev)
+    gbs("rht32_mxfp8", lambda: M.rht32_quantize(pay, 11, M.FMT_MXFP8, pc8, ps8), Rr * d, 3.03125)
+    del pay, pc8, ps8
+    # MXFP8 backward operands on the permuted, per-expert padded layout
+    off = L["off"].cpu().numpy()
+    tok = L["tok"].cpu().numpy()
+    Rp = int(off[-1])
+    pad = torch.from_numpy(tok[:Rp] < 0).to(dev)
+    dchans = synth.outlier_channels(7, d, max(1, d // 1000))
+    dy = synth.grad_rows_torch(7, 0, Rp, d, dchans, dev)
+    dy[pad] = 0
+    act = synth.rows_torch(8, synth.TAG_ACT, 0, Rp, f, 0.3, dev)
+    act[pad] = 0
+    dyc0 = torch.empty(Rp, d, dtype=torch.uint8, device=dev)
+    dys0 = torch.empty(Rp * d // 32, dtype=torch.uint8, device=dev)
+    dyc1 = torch.empty(d, Rp, dtype=torch.uint8, device=dev)
+    dys1 = torch.empty(d * Rp // 32, dtype=torch.uint8, device=dev)
+    gbs("mxfp8_sr_rows", lambda: M.mxfp8_quantize_sr(dy, dyc0, dys0, axis=0, seed=7, offset=0,
+                                                     layout=M.LAYOUT_MMA), Rp * d, 3.03125)
+    gbs("mxfp8_sr_cols", lambda: M.mxfp8_quantize_sr(dy, dyc1, dys1, axis=1, seed=7, offset=1,
+                                                     layout=M.LAYOUT_MMA), Rp * d, 3.03125)
+    ac1 = torch.empty(f, Rp, dtype=torch.uint8, device=dev)
+    as1 = torch.empty(f * Rp // 32, dtype=torch.uint8, device=dev)
+    M.mxfp8_quantize_sr(act, ac1, as1, axis=1, rounding=M.ROUND_RNE, layout=M.LAYOUT_MMA)
+    # W2^T per expert, blocks along d (the dgrad contraction), RNE
+    w2c = torch.empty(E * f, d, dtype=torch.uint8, device=dev)
+    w2s = torch.empty(E * f * d // 32, dtype=torch.uint8, device=dev)
+    for e in range(E):
+        wb = synth.expert_weight_torch(1, synth.TAG_W2, e, d, f, dev)
+        M.mxfp8_quantize_sr(wb, w2c[e * f:(e + 1) * f], w2s[e * f * d // 32:(e + 1) * f * d // 32],
+                            axis=1, rounding=M.ROUND_RNE, layout=M.LAYOUT_MMA)
+    del wb
+    fp8_peak = peaks["bf16_sustained"] * 2.0
+    R_real = T * k
+    flops = 2.0 * R_real * d * f
+    dA = torch.empty(Rp, f, dtype=torch.bfloat16, device=dev)
+    ms = time_kernel(torch, lambda: M.mxfp8_grouped_gemm(dyc0, dys0, w2c, w2s, L["off"], E,
+                                                         M.GROUP_M, Rp, f, d, dA,
+                                                         out_dtype=M.OUT_BF16), reps, flush)
+    res["mxfp8_dgrad_gemm"] = {"ms": round(ms, 4), "TFLOPS": round(flops / ms / 1e9, 1),
+                               "frac_fp8_peak": round(flops / ms / 1e9 / fp8_peak, 3)}
+    del dA
+    dW = torch.empty(E, d, f, dtype=torch.float32, device=dev)
+    ms = time_kernel(torch, lambda: M.mxfp8_grouped_gemm(dyc1, dys1, ac1, as1, L["off"], E,
+                                                         M.GROUP_K, d, f, Rp, dW,
+                                                         out_dtype=M.OUT_F32), reps, flush)
+    res["mxfp8_wgrad_gemm"] = {"ms": round(ms, 4), "TFLOPS": round(flops / ms / 1e9, 1),
+                               "frac_fp8_peak": round(flops / ms / 1e9 / fp8_peak, 3),
+                               "note": "fp32 dW [E x d x f] written"}
+    del dW, dy, act, dyc0, dys0, dyc1, dys1, ac1, as1, w2c, w2s, flush_buf
+    torch.cuda.empty_cache()
+    res["fp8_peak_tflops"] = fp8_peak
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (the baseline; also the --impl reference arm)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """One expert of the full-size layer on the CPU oracle: quantize that
+    expert's routed token rows, GEMM1 + SwiGLU + requantize + GEMM2 in fp64.
+    The weights are quantized once at set-up, like the GPU arm's."""
+
+    def __init__(self, shape, router, expert=0):
+        import oracle as orc
+        from precision_moe_numerics_quantize_b200 import synth
+        self.orc, self.synth = orc, synth
+        T, d, f, E, k = shape.T, shape.d, shape.f, shape.E, shape.k
+        logits = (synth.logits_uniform_np(2, T, E) if router == "uniform"
+                  else synth.logits_zipf_np(2, T, E))
+        idx, _ = orc.route(logits, k)
+        off, pos, tok = orc.permute(idx, E)
+        rows = np.arange(off[expert], off[expert + 1])
+        self.tokens = tok[rows][tok[rows] >= 0]
+        # only the routed rows are generated; the sample is quantized with its own amax
+        self.xrows = np.ascontiguousarray(np.stack([
+            synth.bf16_bits_to_f32(synth.rows_np(0, synth.TAG_X, int(t), 1, d, 1.0))[0]
+            for t in self.tokens]))
+        self.amax = None
+        W1 = synth.bf16_bits_to_f32(synth.expert_weight_np(1, synth.TAG_W1, expert, 2 * f, d))
+        W2 = synth.bf16_bits_to_f32(synth.expert_weight_np(1, synth.TAG_W2, expert, d, f))
+        self.w1 = orc.nvfp4_quantize(W1)
+        self.w2 = orc.nvfp4_quantize(W2)
+        self.d, self.f = d, f
+        self.flops = 6.0 * len(self.tokens) * d * f
+
+    def step(self):
+        xc, xs, xt = self.orc.nvfp4_quantize(self.xrows, amax_in=self.amax)
+        return self.orc.expert_ffn(xc, xs, xt, *self.w1, *self.w2)
+
+    def describe(self):
+        return (f"one expert of the full-size layer: {len(self.tokens)} routed rows x d={self.d}, "
+                f"f={self.f} (x-row quantization + GEMM1 + SwiGLU + requantization + GEMM2)")
+
+
+def cpu_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def run_reference(args, shape):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    s = OracleSample(shape, args.router)
+    for _ in range(args.warmup):
+        s.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s.step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = s.flops / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(args, shape), "sample": s.describe()},
+            "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": cpu_threads(),
+                             "kind": "oracle", "sample": s.describe()},
+            "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_name(args, shape):
+    return (f"{args.workload} router={args.router}: T={shape.T} d={shape.d} f={shape.f} "
+            f"E={shape.E} top-{shape.k} SwiGLU")
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["full_moe", "small_moe"], default="full_moe")
+    ap.add_argument("--router", choices=["uniform", "zipf"], default="uniform")
+    ap.add_argument("--no-companions", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from precision_moe_numerics_quantize_b200 import synth
+    shape = synth.SHAPES[args.workload]
+    if args.impl == "reference":
+        run_reference(args, shape)
+        return
+
+    import torch
+    from precision_moe_numerics_quantize_b200 import build as B
+    B.build()
+    from precision_moe_numerics_quantize_b200 import nvfp4moe as M
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+
+    L = setup_layer(M, synth, torch, dev, shape, args.router)
+    calls = layer_calls(M, L)
+    for _ in range(args.warmup):
+        for _, fn in calls:
+            fn()
+    torch.cuda.synchronize()
+    st, code = M.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error after warm-up: wait id {code}")
+
+    # ---- timed region: K steps, inputs resident ----
+    sampler = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms, per_call = time_calls(torch, calls, args.steps)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = total_ms / args.steps
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    T, d, f, E, k = shape.T, shape.d, shape.f, shape.E, shape.k
+    flops = 6.0 * T * k * d * f
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    stream = torch.cuda.current_stream()
+    ea = torch.cuda.Event(enable_timing=True)
+    eb = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ea.record()
+    for _ in range(args.steps):
+        L["x"].copy_(L["x_host"], non_blocking=True)
+        L["logits"].copy_(L["logits_host"], non_blocking=True)
+        for _, fn in calls:
+            fn()
+        L["out_host"].copy_(L["out"], non_blocking=True)
+    eb.record()
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+           "h2d_bytes_per_step": L["x_host"].numel() * 2 + L["logits_host"].numel() * 4,
+           "d2h_bytes_per_step": L["out_host"].numel() * 2, "ms_per_step": e2e_ms}
+    del stream
+
+    fp4_peak = peaks["bf16_sustained"] * 4.0
+    ex_ms = per_call["moe_expert_fwd"]
+    achieved = flops / (ex_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
+                "traffic": EXPERT_FWD_DRAM_BYTES,
+                "kernel": "moe_expert_fwd (grouped GEMM1+SwiGLU+amax, requantize, grouped GEMM2)",
+                "peak_source": f"{peaks['source']} bf16 sustained x 4 (nominal FP4:BF16 ratio)",
+                "weights_hbm_floor_ms": round(0.5625 * 3 * d * f * E / (peaks["hbm_gbs"] * 1e6), 3)}
+
+    comp = None
+    if rank == 0 and not args.no_companions:
+        comp = companions(M, synth, torch, dev, L, peaks)
+    if dist:
+        dist.barrier()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s = OracleSample(shape, args.router)
+        t0 = time.perf_counter()
+        s.step()
+        dt = time.perf_counter() - t0
+        cpu = {"value": s.flops / dt / 1e12, "unit": "TFLOPS", "cores": cpu_threads(),
+               "kind": "oracle", "sample": s.describe(), "seconds": round(dt, 2)}
+
+    launches = args.steps * sum(KERNELS_PER_STEP.values())
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "nvfp4 (e2m1 x e2m1, fp32 accumulate)", "data": "synthetic",
+                "config": {"workload": workload_name(args, shape), "global_batch": T * world,
+                           "routed_rows_per_gpu": T * k, "parallelism": f"replicas x{world}",
+                           "l2": "inputs larger than L2 (6.8 GB NVFP4 weights per step)",
+                           "per_call_ms": {n: round(v, 4) for n, v in per_call.items()}},
+                "fp4_peak_frac": round(value / world / fp4_peak, 4),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clocks, "companions": comp}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,278 @@
+/*
+ * nvfp4moe: NVFP4 mixture-of-experts expert layer for NVIDIA B200 (sm_100a).
+ *
+ * The method: write-ups of Thinking Machines Lab's "End-to-End 4-Bit
+ * Training" post.
+ *   - news.t0001.com, "Thinking Machines 详解 Inkling 2 Small 原生 4-bit 前向训练完整流程",
+ *     list "训练数值格式分工清单": expert-layer forward passes in NVFP4 on
+ *     dedicated CUDA kernels, backward gradients in MXFP8 with stochastic
+ *     rounding, quantized cross-GPU traffic, non-expert modules at higher
+ *     precision.
+ *   - aicoder.com, "Thinking Machines Details End-to-End 4-Bit Training for
+ *     Inkling 2 Small", "Key Takeaways" and "Architecture highlights": MXFP8
+ *     backward with re-quantization and stochastic rounding; the
+ *     expert-parallel combine is quantized after a 32-dimensional random
+ *     Hadamard transform into a block-scaled format; the kernels are fully
+ *     deterministic. "Background": NVFP4 costs about 4.5 bits per value.
+ *   - 10100.com, "Inkling 2 Small", "PART 01": 384 experts, top-8 routing.
+ * The pages print no formula. The numeric readings this library implements:
+ *   NVFP4  = E2M1 codes (grid 0, .5, 1, 1.5, 2, 3, 4, 6; nearest, ties to even,
+ *            saturating), one E4M3 scale per 16 elements, one fp32 decode
+ *            scale per tensor: ts = amax / 2688, S_enc = 2688 / amax,
+ *            s_b = E4M3_RNE((amax_b / 6) * S_enc), q = E2M1_RNE(x * S_enc / s_b),
+ *            x_hat = e2m1(q) * s_b * ts (amax 0 -> S_enc = ts = 1).
+ *   MXFP8  = E4M3 codes, one E8M0 scale 2^k per 32 elements, k the smallest
+ *            integer in [-127, 127] with amax_b <= 448 * 2^k (nothing clips);
+ *            rounding to nearest even, or stochastic with Philox4x32-10
+ *            (key = seed, counter = (i / 4, offset), word i % 4, i the
+ *            row-major index of the element in the source tensor): round up
+ *            iff (word >> 8) * 2^-24 < (|v| - lo) / (hi - lo).
+ *   RHT32  = v = fp32(1/sqrt(32)) * H32 * (s .* x) per 32-element block; H32
+ *            Sylvester; s_i = -1 iff bit i of word 0 of Philox4x32-10(key =
+ *            sign_seed, counter = 0); fp32 butterflies h = 1, 2, 4, 8, 16.
+ *
+ * Conventions (all entry points):
+ *   - Every function returns an nvfp4moe_status. Arguments are validated on
+ *     the host before anything is launched; a failed validation leaves every
+ *     output untouched. NVFP4MOE_ERR_CUDA carries the CUDA error text in
+ *     nvfp4moe_last_error() (thread-local).
+ *   - All pointers named in a signature are DEVICE pointers unless the comment
+ *     says "host". The caller owns all memory; the library allocates nothing.
+ *     Tensor pointers (bf16 data, codes, scales, outputs, workspace) must be
+ *     16-byte aligned; fp32 scalars (amax, ts) and int32 index arrays
+ *     4-byte aligned (NVFP4MOE_ERR_ALIGN).
+ *   - Every call is asynchronous on the given stream, performs no host
+ *     synchronisation, and is deterministic (identical bits for identical
+ *     inputs). The one piece of library state is a device-side error word
+ *     set by a kernel whose bounded wait ran out; nvfp4moe_device_error()
+ *     reads and clears it.
+ *   - bf16 tensors are passed as uint16_t bit patterns, row-major, with a row
+ *     stride ld in elements (ld >= cols, ld % 8 == 0).
+ *   - NVFP4 codes: rows x cols/2 bytes, element 2i in the low nibble of byte i.
+ *   - Scale layouts:
+ *       NVFP4MOE_LAYOUT_ROWMAJOR: scales[r * (cols / B) + b] (B = 16 or 32).
+ *       NVFP4MOE_LAYOUT_MMA: the tcgen05 block-scaled MMA layout. Scales are
+ *         grouped in 512-byte chunks, one per 128 rows x 4 scale columns;
+ *         chunk (rt, kc) starts at byte (rt * (cols / B / 4) + kc) * 512 and
+ *         the scale of row r = 128 rt + 32 r1 + r0 (r0 < 32, r1 < 4) and scale
+ *         column 4 kc + c sits at byte r0 * 16 + r1 * 4 + c of its chunk.
+ *         Needs rows % 128 == 0 and (cols / B) % 4 == 0.
+ */
+#ifndef NVFP4MOE_H
+#define NVFP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The library is built with hidden visibility; the entry points below are
+ * the only exported symbols. */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef struct CUstream_st *nvfp4moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    NVFP4MOE_OK = 0,
+    NVFP4MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, k > E, bad enum, aliasing */
+    NVFP4MOE_ERR_SHAPE = 2,       /* a dimension breaks the divisibility rule of the call */
+    NVFP4MOE_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+    NVFP4MOE_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query says */
+    NVFP4MOE_ERR_CUDA = 5,        /* a CUDA call failed; see nvfp4moe_last_error() */
+    NVFP4MOE_ERR_TIMEOUT = 6,     /* a bounded device wait ran out (nvfp4moe_device_error) */
+    NVFP4MOE_ERR_UNSUPPORTED = 7  /* valid request this build does not implement */
+} nvfp4moe_status;
+
+enum { NVFP4MOE_LAYOUT_ROWMAJOR = 0, NVFP4MOE_LAYOUT_MMA = 1 };
+enum { NVFP4MOE_ROUND_RNE = 0, NVFP4MOE_ROUND_SR = 1 };
+enum { NVFP4MOE_FMT_NVFP4 = 0, NVFP4MOE_FMT_MXFP8 = 1 };
+enum { NVFP4MOE_OUT_BF16 = 0, NVFP4MOE_OUT_F32 = 1 };
+enum { NVFP4MOE_GROUP_M = 0, NVFP4MOE_GROUP_K = 1 };
+
+/* Library version, e.g. 100 for 0.1.0. */
+int nvfp4moe_version(void);
+
+/* Text of the last error on this thread ("" if none). Owned by the library. */
+const char *nvfp4moe_last_error(void);
+
+/* Synchronises the current device, then reads and clears the device error
+ * word. *code (host) receives 0 if no kernel gave up a bounded wait, else the
+ * identifier of the wait that ran out. Returns NVFP4MOE_ERR_TIMEOUT if set. */
+nvfp4moe_status nvfp4moe_device_error(int32_t *code);
+
+/* Upper bound on the rows of a permuted, per-expert-padded activation:
+ * T*k + E*127 rounded up to 128. Pure host arithmetic. */
+int64_t nvfp4moe_max_rows(int64_t T, int32_t k, int32_t E);
+
+/* ------------------------------------------------------------------------
+ * max |x| over a bf16 tensor (the NVFP4 tensor amax).
+ * x [rows x cols], stride ld. amax: one fp32, overwritten. */
+nvfp4moe_status nvfp4moe_amax_bf16(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                   float *amax, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * NVFP4 quantization (news.t0001.com '训练数值格式分工清单': the expert forward in
+ * NVFP4; aicoder.com 'Background': about 4.5 bits per value).
+ * x: bf16 [rows x cols], stride ld; cols % 64 == 0.
+ * amax_in: device fp32 or NULL. NULL computes max|x| first (two passes);
+ *   a caller that already holds the amax passes it (one pass). Must not
+ *   alias ts_out.
+ * codes: [rows x cols/2]. scales: E4M3 in `layout`. ts_out: one fp32, the
+ *   decode tensor scale amax / 2688. */
+nvfp4moe_status nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                               const float *amax_in, uint8_t *codes, uint8_t *scales,
+                               float *ts_out, int layout, nvfp4moe_stream_t stream);
+
+/* out[r][c] = e2m1(code) * scale * ts in fp32, out [rows x cols] fp32.
+ * ts: device fp32 (one value). */
+nvfp4moe_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                 int64_t rows, int64_t cols, int layout, float *out,
+                                 nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * MXFP8 quantization with stochastic rounding (news.t0001.com '训练数值格式分工清单':
+ * MXFP8 backward with stochastic rounding; aicoder.com 'Key Takeaways':
+ * re-quantization and stochastic rounding to limit gradient bias).
+ * x: bf16 [rows x cols], stride ld.
+ * axis 0: blocks of 32 along a row. cols % 32 == 0 (MMA layout: rows % 128,
+ *   cols % 128). codes [rows x cols], scales E8M0 [rows x cols/32].
+ * axis 1: blocks of 32 consecutive rows of a column; rows % 32 == 0 (MMA:
+ *   rows % 128, cols % 128). The output is transposed, ready to be the
+ *   K-major operand of a GEMM that contracts over rows: codes [cols x rows],
+ *   scales [cols x rows/32]. To keep blocks inside expert segments, start
+ *   every segment on a 32-row boundary (moe_route_permute pads to 128).
+ * rounding: NVFP4MOE_ROUND_RNE or NVFP4MOE_ROUND_SR (seed, offset select the
+ *   Philox stream; quantize the same tensor along two axes with two offsets). */
+nvfp4moe_status mxfp8_quantize_sr(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                  int axis, uint64_t seed, uint64_t offset, int rounding,
+                                  uint8_t *codes, uint8_t *scales, int layout,
+                                  nvfp4moe_stream_t stream);
+
+/* out = e4m3(code) * 2^(scale - 127), fp32 [n_rows x n_cols] for an MXFP8
+ * tensor stored as codes [n_rows x n_cols] with ROWMAJOR or MMA scales. */
+nvfp4moe_status mxfp8_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t n_rows,
+                                 int64_t n_cols, int layout, float *out,
+                                 nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * RHT32 + block-scaled quantization of the combine payload (aicoder.com 'Key
+ * Takeaways' and 'Architecture highlights': a 32-dimensional random Hadamard
+ * transform before the expert-parallel combine traffic is quantized).
+ * x: bf16 [rows x cols], stride ld, cols % 32 == 0. ROWMAJOR scales only.
+ * fmt NVFP4: codes [rows x cols/2], scales [rows x cols/16], ts_out (decode
+ *   tensor scale of the transformed values; amax_in as in nvfp4_quantize,
+ *   but the amax of the TRANSFORMED values).
+ * fmt MXFP8 (round to nearest even): codes [rows x cols], scales
+ *   [rows x cols/32]; amax_in and ts_out unused (may be NULL). */
+nvfp4moe_status rht32_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                               uint64_t sign_seed, int fmt, const float *amax_in,
+                               uint8_t *codes, uint8_t *scales, float *ts_out, int layout,
+                               nvfp4moe_stream_t stream);
+
+/* Inverse: dequantize, inverse transform; out fp32 [rows x cols]. ts: device
+ * fp32 for NVFP4 (ignored for MXFP8). */
+nvfp4moe_status rht32_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                 int64_t rows, int64_t cols, uint64_t sign_seed, int fmt,
+                                 int layout, float *out, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Routing and dispatch with fused NVFP4 quantization (10100.com 'PART 01':
+ * top-8 of 384 experts; aicoder.com 'Key Takeaways': expert-parallel
+ * dispatch and combine).
+ * logits fp32 [T x E]; x bf16 [T x d] (ld = d). 1 <= k <= min(E, 32),
+ * E <= 1024, d % 64 == 0.
+ * Top-k by logit (largest first, ties to the lower expert id). renorm = 1:
+ * weights = softmax over the k chosen logits (= p_j / sum of chosen p);
+ * renorm = 0: weights = softmax over all E.
+ * Slots (t, j) are grouped by expert, ascending (t, j) inside an expert, each
+ * expert's rows start at a multiple of 128.
+ * Outputs: topk_idx int32 [T x k], topk_w fp32 [T x k], expert_off int32
+ *   [E + 1] (expert_off[E] = used rows), pos int32 [T x k] (slot -> row),
+ *   token_of int32 [R] (row -> token, -1 for a padding row),
+ *   xq [R x d/2] and xq_sc (MMA layout, R rows) = NVFP4 of x with one tensor
+ *   scale for all of x, padding rows zero; x_ts (one fp32).
+ *   R = nvfp4moe_max_rows(T, k, E); rows >= expert_off[E] are not written
+ *   except token_of (-1).
+ * x_amax_in: device fp32 or NULL (NULL: computed here).
+ * ws: device workspace of at least moe_route_permute_workspace_size() bytes. */
+size_t moe_route_permute_workspace_size(int64_t T, int32_t E, int32_t k);
+nvfp4moe_status moe_route_permute(const float *logits, const uint16_t *x, int64_t T, int32_t E,
+                                  int32_t k, int64_t d, int renorm, const float *x_amax_in,
+                                  int32_t *topk_idx, float *topk_w, int32_t *expert_off,
+                                  int32_t *pos, int32_t *token_of, uint8_t *xq, uint8_t *xq_sc,
+                                  float *x_ts, void *ws, size_t ws_bytes,
+                                  nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert FFN forward in NVFP4 (news.t0001.com '训练数值格式分工清单'; aicoder.com
+ * 'Architecture highlights': NVFP4 forward in the expert layers).
+ * For every expert e, rows [expert_off[e], expert_off[e+1]):
+ *   [g | u] = dq(xq) . dq(W1_e)^T in fp32 on the tensor cores,
+ *   h       = bf16(silu(g) * u),            silu(g) = g / (1 + exp(-g))
+ *   h_amax[e] = max |h| over the expert's rows,
+ *   hq      = NVFP4(h) with the per-expert tensor scale h_ts[e] = h_amax[e] / 2688,
+ *   y       = bf16(dq(hq) . dq(W2_e)^T).
+ * xq [R x d/2], xq_sc (MMA), x_ts (one fp32): from moe_route_permute.
+ * w1 [E x 2f x d/2] codes, w1_sc MMA layout of the [E*2f x d] matrix, w1_ts
+ *   fp32 [E]; rows 0..f-1 of W1_e give g, rows f..2f-1 give u.
+ * w2 [E x d x f/2], w2_sc MMA layout of [E*d x f], w2_ts fp32 [E].
+ *   (Quantize each expert with nvfp4_quantize, MMA layout, its own amax.)
+ * Caller-provided intermediates (outputs too): h bf16 [R x f], hq [R x f/2],
+ *   hq_sc MMA layout of [R x f], h_amax fp32 [E], h_ts fp32 [E].
+ * y bf16 [R x d]. R = rows_alloc >= expert_off[E], R % 128 == 0.
+ * d % 256 == 0, f % 256 == 0, E <= 1024. */
+nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const float *x_ts,
+                               const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
+                               const uint8_t *w1, const uint8_t *w1_sc, const float *w1_ts,
+                               const uint8_t *w2, const uint8_t *w2_sc, const float *w2_ts,
+                               uint16_t *h, uint8_t *hq, uint8_t *hq_sc, float *h_amax,
+                               float *h_ts, uint16_t *y, int64_t rows_alloc,
+                               nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Weighted top-k combine (aicoder.com 'Key Takeaways': the combine step).
+ * out[t] = bf16( sum_{j=0..k-1} topk_w[t,j] * y[pos[t,j]] ), fp32 accumulation
+ * in slot order with fused multiply-adds; a gather, no atomics.
+ * y bf16 [* x d] (row stride d); pos, topk_w [T x k]; out bf16 [T x d].
+ * d % 8 == 0. */
+nvfp4moe_status moe_combine(const uint16_t *y, const int32_t *pos, const float *topk_w,
+                            int64_t T, int32_t k, int64_t d, uint16_t *out,
+                            nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped block-scaled GEMMs on the tcgen05 tensor cores.
+ *
+ * nvfp4_grouped_gemm: for every group g, rows [off[g], off[g+1]) of A
+ *   (multiples of 128):  C[rows] = alpha_g * dq(A[rows]) . dq(B_g)^T with
+ *   alpha_g = a_ts[g * a_ts_stride] * b_ts[g], fp32 accumulation.
+ *   A [R x K/2] NVFP4 + MMA scales; B [G x N x K/2] + MMA scales of [G*N x K];
+ *   C [R x N] bf16 or fp32 (out_dtype), row stride N. K % 256 == 0,
+ *   N % 256 == 0, G <= 1024, R % 128 == 0.
+ * mxfp8_grouped_gemm: E4M3 x E4M3 with E8M0 scales (MMA layout), fp32 accumulation.
+ *   group_axis M: as above with A [R x K], B [G x N x K], C [R x N].
+ *   group_axis K: group g contracts over columns [off[g], off[g+1]) of
+ *     A [M x Kt] and B [N x Kt] (offsets multiples of 128) into C_g [M x N];
+ *     C [G x M x N] (a group with no columns writes zeros). M % 128 == 0.
+ *   K % 128 == 0 (group M), N % 256 == 0. */
+nvfp4moe_status nvfp4_grouped_gemm(const uint8_t *a, const uint8_t *a_sc, const float *a_ts,
+                                   int32_t a_ts_stride, const uint8_t *b, const uint8_t *b_sc,
+                                   const float *b_ts, const int32_t *group_off, int32_t G,
+                                   int64_t R, int64_t N, int64_t K, void *c, int out_dtype,
+                                   nvfp4moe_stream_t stream);
+nvfp4moe_status mxfp8_grouped_gemm(const uint8_t *a, const uint8_t *a_sc, const uint8_t *b,
+                                   const uint8_t *b_sc, const int32_t *group_off, int32_t G,
+                                   int group_axis, int64_t M, int64_t N, int64_t K, void *c,
+                                   int out_dtype, nvfp4moe_stream_t stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4MOE_H */

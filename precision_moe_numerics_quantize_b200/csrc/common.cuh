@@ -1,0 +1,349 @@
+// Device-side building blocks shared by the nvfp4moe kernels: status
+// plumbing, bf16 loads, the E2M1 / E4M3 / E8M0 encoders, Philox4x32-10, and
+// thin inline-PTX wrappers for mbarriers, TMA and tcgen05 (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nvfp4moe.h"
+
+#define NV_DEV __device__ __forceinline__
+
+namespace nvfp4moe {
+
+// ---------------------------------------------------------------------------
+// host-side error plumbing (defined in abi.cu)
+// ---------------------------------------------------------------------------
+void set_last_error(const char *fmt, ...);
+nvfp4moe_status cuda_status(cudaError_t e, const char *what);
+
+// Device error word: a kernel whose bounded wait ran out stores the id of the
+// wait here (first writer wins) and returns early.
+extern __device__ int32_t g_device_error;
+
+enum WaitId : int32_t {
+    WAIT_NONE = 0,
+    WAIT_GEMM_FULL = 1,
+    WAIT_GEMM_EMPTY = 2,
+    WAIT_GEMM_ACC_FULL = 3,
+    WAIT_GEMM_ACC_EMPTY = 4,
+    WAIT_GEMM_DRAIN = 5,
+};
+
+// ---------------------------------------------------------------------------
+// small helpers
+// ---------------------------------------------------------------------------
+NV_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+NV_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// fp32 -> bf16 bits, nearest with ties to even (finite inputs; NaN -> quiet NaN).
+NV_DEV uint32_t f32_to_bf16_bits(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return 0x7FC0u;
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return u >> 16;
+}
+
+NV_DEV float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// Non-negative floats order like their bit patterns: max via unsigned atomics.
+NV_DEV void atomic_max_nonneg(float *addr, float v) {
+    atomicMax(reinterpret_cast<unsigned int *>(addr), __float_as_uint(v));
+}
+
+// ---------------------------------------------------------------------------
+// E2M1: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}. Nearest value, ties to the
+// even code, saturating; the sign bit is the input's sign. The decision
+// points are the midpoints between neighbouring magnitudes; a midpoint goes
+// to the neighbour with the even code.
+// ---------------------------------------------------------------------------
+NV_DEV uint32_t e2m1_encode(float v) {
+    float a = fabsf(v);
+    uint32_t m = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+                 (a >= 3.5f) + (a > 5.0f);
+    return m | ((__float_as_uint(v) >> 28) & 8u);
+}
+
+NV_DEV float e2m1_decode(uint32_t nib) {
+    // magnitude m: 0..3 -> m/2, 4 -> 2, 5 -> 3, 6 -> 4, 7 -> 6
+    uint32_t m = nib & 7u;
+    float mag = (m < 4u) ? 0.5f * (float)m : (m == 7u ? 6.0f : (float)(m - 2u));
+    return (nib & 8u) ? -mag : mag;
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 (bias 7, max 448, no infinities). Encoding of a non-negative finite
+// value: nearest, ties to even, saturating at 448.
+//   a >= 448         -> 0x7E
+//   a <  2^-6        -> subnormal: mantissa = round(a * 2^9) (0..8; 8 is 2^-6)
+//   otherwise        -> exponent e = floor(log2 a) from the fp32 exponent
+//                       field, 3-bit mantissa rounded from the 23-bit one.
+// ---------------------------------------------------------------------------
+NV_DEV uint32_t e4m3_encode_pos(float a) {
+    if (a >= 448.0f) return 0x7Eu;
+    if (a < 0.015625f) return (uint32_t)__float2int_rn(a * 512.0f);
+    uint32_t u = __float_as_uint(a);
+    int e = (int)((u >> 23) & 0xFF) - 127;  // -6 .. 8
+    uint32_t man = u & 0x7FFFFFu;
+    uint32_t m3 = man >> 20, rem = man & 0xFFFFFu;
+    uint32_t code = ((uint32_t)(e + 7) << 3) | m3;
+    if (rem > 0x80000u || (rem == 0x80000u && (m3 & 1u))) code += 1u;
+    return code;
+}
+
+NV_DEV uint32_t e4m3_encode(float v) {
+    return e4m3_encode_pos(fabsf(v)) | ((__float_as_uint(v) >> 24) & 0x80u);
+}
+
+NV_DEV float e4m3_decode_pos(uint32_t c) {  // c in 0..126
+    uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    if (e == 0) return (float)m * 0.001953125f;  // m * 2^-9
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+NV_DEV float e4m3_decode(uint32_t c) {
+    float v = e4m3_decode_pos(c & 0x7Fu);
+    return (c & 0x80u) ? -v : v;
+}
+
+// 2^e as an fp32 for e in [-126, 127].
+NV_DEV float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// ---------------------------------------------------------------------------
+// MXFP8 block exponent: smallest k in [-127, 127] with amax <= 448 * 2^k.
+// amax = m * 2^E (m in [1, 2)); 448 = 1.75 * 2^8: k = E - 8 if m <= 1.75,
+// else E - 7. Zero and subnormal amax clamp to -127.
+// ---------------------------------------------------------------------------
+NV_DEV int mx_scale_exp(float amax) {
+    uint32_t u = __float_as_uint(amax);
+    int ef = (int)((u >> 23) & 0xFF);
+    if (ef == 0) return -127;
+    int E = ef - 127;
+    uint32_t man = u & 0x7FFFFFu;
+    int k = (man <= 0x600000u) ? E - 8 : E - 7;  // 0x600000 = 0.75 * 2^23
+    return k < -127 ? -127 : (k > 127 ? 127 : k);
+}
+
+// v * 2^-k exactly (k in [-127, 127]).
+NV_DEV float scale_pow2(float v, int k) {
+    int nk = -k;
+    if (nk > 127) return (v * exp2i(127)) * exp2i(nk - 127);
+    if (nk < -126) return (v * exp2i(-126)) * exp2i(nk + 126);
+    return v * exp2i(nk);
+}
+
+// E4M3 code of v with stochastic rounding driven by the 32-bit word r:
+// E4M3 spacing q = 2^(max(floor(log2|v|), -6) - 3); with lo = floor(|v|/q)*q,
+// round up iff (r >> 8) * 2^-24 < (|v| - lo) / q. |v| <= 448 is assumed.
+NV_DEV uint32_t e4m3_encode_sr(float v, uint32_t r) {
+    float a = fabsf(v);
+    uint32_t u = __float_as_uint(a);
+    int e = (int)((u >> 23) & 0xFF) - 127;
+    if (e < -6) e = -6;
+    float inv_q = exp2i(3 - e);       // 1/q, exact
+    float m = a * inv_q;              // exact: |v| has at most 24 significant bits
+    float lo = floorf(m);
+    float frac = m - lo;              // exact
+    float rr = (float)(r >> 8) * 5.9604644775390625e-08f;  // r * 2^-24, exact
+    float mag = (rr < frac) ? lo + 1.0f : lo;
+    float res = mag * exp2i(e - 3);   // exact
+    return e4m3_encode_pos(res) | ((__float_as_uint(v) >> 24) & 0x80u);
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11): 10 rounds of the multiply-xor bijection
+// with the published multipliers and Weyl key increments.
+// ---------------------------------------------------------------------------
+struct u32x4 { uint32_t x, y, z, w; };
+
+NV_DEV u32x4 philox4x32_10(u32x4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int i = 0; i < 10; ++i) {
+        uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = u32x4{hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0};
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c;
+}
+
+// The four words for elements 4*blk .. 4*blk+3 of the (seed, offset) stream.
+NV_DEV u32x4 philox_block(uint64_t seed, uint64_t offset, uint64_t blk) {
+    return philox4x32_10(u32x4{(uint32_t)blk, (uint32_t)(blk >> 32), (uint32_t)offset,
+                               (uint32_t)(offset >> 32)},
+                         (uint32_t)seed, (uint32_t)(seed >> 32));
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers: shared-memory addresses, mbarriers, TMA, tcgen05.
+// ---------------------------------------------------------------------------
+NV_DEV uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+NV_DEV void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+NV_DEV void fence_mbarrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+NV_DEV void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+NV_DEV void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+NV_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+NV_DEV uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase with the given parity to complete, giving up after about
+// two seconds: on timeout the wait id goes to the device error word and the
+// caller returns false so the kernel can wind down instead of hanging.
+NV_DEV bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int32_t wait_id) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > 2000000000ull) {
+            atomicCAS(&g_device_error, 0, wait_id);
+            return false;
+        }
+    }
+}
+
+// TMA tiled 2D load into shared memory, completion counted on an mbarrier.
+NV_DEV void tma_load_2d(void *dst, const CUtensorMap *map, int32_t x, int32_t y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Plain bulk copy global -> shared (16-byte aligned, size % 16 == 0).
+NV_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+NV_DEV void prefetch_tmap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// --- tcgen05 ---------------------------------------------------------------
+NV_DEV void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+NV_DEV void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+NV_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+NV_DEV void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+NV_DEV void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive on an mbarrier once every previously issued tcgen05 op of this thread completes.
+NV_DEV void tc_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+// Copy a 32-row x 128-bit block from shared memory into TMEM, replicated to
+// all four 32-lane sub-partitions.
+NV_DEV void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+NV_DEV void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+        "[%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+NV_DEV void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], "
+        "p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.
+NV_DEV void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+NV_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (tcgen05 format): start address, leading and
+// stride byte offsets in 16-byte units, descriptor version 1 (bit 46), swizzle
+// mode in bits 61..63 (0 none, 2 = 128-byte swizzle).
+NV_DEV uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                          uint32_t swizzle) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)(swizzle & 7u) << 61;
+    return d;
+}
+
+}  // namespace nvfp4moe

@@ -1,0 +1,596 @@
+// Bandwidth-bound quantizers: tensor amax, NVFP4 (16-element E4M3-scaled
+// E2M1), MXFP8 (32-element E8M0-scaled E4M3, nearest or Philox stochastic
+// rounding, along rows or along columns), and the 32-point random Hadamard
+// transform followed by block-scaled quantization of the combine payload.
+//
+// Every kernel reads its input with 16-byte vector loads in a coalesced
+// pattern and writes codes with 16-byte stores; scales are written either
+// row-major or directly in the tcgen05 MMA layout (512-byte chunks of
+// 128 rows x 4 scales) so that the GEMMs can stream them with bulk copies.
+#include "common.cuh"
+#include "quant.cuh"
+
+namespace nvfp4moe {
+
+__device__ int32_t g_device_error = 0;
+
+// Byte offset of scale (row r, scale column c) in the MMA layout of a matrix
+// whose rows carry `nsc` scales (nsc % 4 == 0).
+NV_DEV size_t mma_sf_offset(int64_t r, int64_t c, int64_t nsc) {
+    int64_t chunk = (r >> 7) * (nsc >> 2) + (c >> 2);
+    return (size_t)chunk * 512 + (size_t)((r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3));
+}
+
+// ---------------------------------------------------------------------------
+// amax of a bf16 tensor. *amax must be zero before the launch.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const uint16_t *__restrict__ x,
+                                                        int64_t rows, int64_t cols, int64_t ld,
+                                                        float *__restrict__ amax) {
+    const int64_t vpr = cols / 8;  // 16-byte vectors per row
+    const int64_t nvec = rows * vpr;
+    float m = 0.0f;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / vpr, c = i - r * vpr;
+        uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + r * ld) + c);
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
+                           fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))),
+                           fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+    }
+    m = warp_max(m);
+    __shared__ float red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+        v = warp_max(v);
+        if (threadIdx.x == 0) atomic_max_nonneg(amax, v);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4: per-tensor S_enc from amax; one thread quantizes 64 consecutive
+// elements (4 blocks of 16): 128 bytes in, 32 bytes of codes and 4 scales out.
+// ---------------------------------------------------------------------------
+NV_DEV float nvfp4_senc(float amax) {
+    return (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(2688.0f, amax) : 1.0f;
+}
+NV_DEV float nvfp4_ts(float amax) {
+    return (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// Quantize 16 fp32 values: returns the scale code, writes 8 code bytes (2 words).
+NV_DEV uint32_t nvfp4_block16(const float (&v)[16], float S_enc, uint32_t &w0, uint32_t &w1) {
+    float amax_b = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+    float t = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S_enc);
+    uint32_t sc = e4m3_encode_pos(t);
+    float sf = e4m3_decode_pos(sc);
+    float enc = (sf == 0.0f) ? 0.0f : __fdiv_rn(S_enc, sf);
+    w0 = 0;
+    w1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w0 |= e2m1_encode(__fmul_rn(v[i], enc)) << (4 * i);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w1 |= e2m1_encode(__fmul_rn(v[8 + i], enc)) << (4 * i);
+    return sc;
+}
+
+NV_DEV void unpack8(uint4 q, float *f) {
+    f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x); f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
+    f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z); f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
+}
+
+// 64 bf16 elements at p -> 32 code bytes at out_codes, 4 scale codes packed in a word.
+NV_DEV uint32_t nvfp4_quant64(const uint16_t *__restrict__ p, float S_enc, uint4 &c0, uint4 &c1) {
+    const uint4 *pv = reinterpret_cast<const uint4 *>(p);
+    uint32_t scw = 0;
+    uint32_t w[8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        float v[16];
+        unpack8(__ldg(pv + 2 * b), v);
+        unpack8(__ldg(pv + 2 * b + 1), v + 8);
+        uint32_t sc = nvfp4_block16(v, S_enc, w[2 * b], w[2 * b + 1]);
+        scw |= sc << (8 * b);
+    }
+    c0 = make_uint4(w[0], w[1], w[2], w[3]);
+    c1 = make_uint4(w[4], w[5], w[6], w[7]);
+    return scw;
+}
+
+__global__ void __launch_bounds__(256) nvfp4_quant_kernel(
+    const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    const float *__restrict__ amax_p, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+    float *__restrict__ ts_out, int layout) {
+    const float amax = *amax_p;
+    const float S_enc = nvfp4_senc(amax);
+    const int64_t G = cols / 64;
+    const int64_t n = rows * G;
+    if (ts_out && blockIdx.x == 0 && threadIdx.x == 0) *ts_out = nvfp4_ts(amax);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, g = i - r * G;
+        uint4 c0, c1;
+        uint32_t scw = nvfp4_quant64(x + r * ld + g * 64, S_enc, c0, c1);
+        uint4 *co = reinterpret_cast<uint4 *>(codes + r * (cols / 2) + g * 32);
+        co[0] = c0;
+        co[1] = c1;
+        if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
+            *reinterpret_cast<uint32_t *>(scales + r * (cols / 16) + g * 4) = scw;
+        else
+            *reinterpret_cast<uint32_t *>(scales + mma_sf_offset(r, g * 4, cols / 16)) = scw;
+    }
+}
+
+// Writes ts = amax / 2688 after a two-pass quantization.
+__global__ void nvfp4_finalize_ts_kernel(float *ts_inout) {
+    *ts_inout = nvfp4_ts(*ts_inout);
+}
+
+__global__ void __launch_bounds__(256) nvfp4_dequant_kernel(
+    const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+    const float *__restrict__ ts_p, int64_t rows, int64_t cols, int layout,
+    float *__restrict__ out) {
+    const float ts = *ts_p;
+    const int64_t G = cols / 16;
+    const int64_t n = rows * G;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, b = i - r * G;
+        uint32_t sc = layout == NVFP4MOE_LAYOUT_ROWMAJOR ? scales[r * G + b]
+                                                         : scales[mma_sf_offset(r, b, G)];
+        float sf = e4m3_decode(sc);
+        uint2 q = *reinterpret_cast<const uint2 *>(codes + r * (cols / 2) + b * 8);
+        float o[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = __fmul_rn(e2m1_decode((q.x >> (4 * j)) & 15u) * sf, ts);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            o[8 + j] = __fmul_rn(e2m1_decode((q.y >> (4 * j)) & 15u) * sf, ts);
+        float4 *op = reinterpret_cast<float4 *>(out + r * cols + b * 16);
+        op[0] = make_float4(o[0], o[1], o[2], o[3]);
+        op[1] = make_float4(o[4], o[5], o[6], o[7]);
+        op[2] = make_float4(o[8], o[9], o[10], o[11]);
+        op[3] = make_float4(o[12], o[13], o[14], o[15]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8 along rows: one thread per 128 consecutive elements of a row (4 blocks).
+// ---------------------------------------------------------------------------
+template <bool SR>
+NV_DEV uint32_t mx_block32(const float (&v)[32], uint64_t seed, uint64_t offset, uint64_t idx0,
+                           uint32_t (&w)[8]) {
+    float amax_b = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+    int k = mx_scale_exp(amax_b);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        uint32_t word = 0;
+        if (SR) {
+            // idx0 is a multiple of 4 here (cols % 32 == 0): one Philox call per 4 elements
+            u32x4 r = philox_block(seed, offset, (idx0 >> 2) + q);
+            uint32_t rs[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                word |= e4m3_encode_sr(scale_pow2(v[4 * q + j], k), rs[j]) << (8 * j);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) word |= e4m3_encode(scale_pow2(v[4 * q + j], k)) << (8 * j);
+        }
+        w[q] = word;
+    }
+    return (uint32_t)(k + 127);
+}
+
+template <bool SR>
+__global__ void __launch_bounds__(256) mxfp8_rows_kernel(
+    const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
+    uint64_t offset, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int layout) {
+    const int64_t G = cols / 32;  // blocks per row
+    const int64_t n = rows * G;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, b = i - r * G;
+        const uint4 *pv = reinterpret_cast<const uint4 *>(x + r * ld + b * 32);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) unpack8(__ldg(pv + j), v + 8 * j);
+        uint32_t w[8];
+        uint32_t sc = mx_block32<SR>(v, seed, offset, (uint64_t)(r * cols + b * 32), w);
+        uint4 *co = reinterpret_cast<uint4 *>(codes + r * cols + b * 32);
+        co[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        co[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
+            scales[r * G + b] = (uint8_t)sc;
+        else
+            scales[mma_sf_offset(r, b, G)] = (uint8_t)sc;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8 along columns, transposed output. A CTA stages a 128-row x 64-column
+// tile in shared memory with coalesced 16-byte loads; thread t quantizes the
+// 32-row block (t / 64) of column (t % 64) and writes its 32 codes as a row
+// of the transposed output.
+// ---------------------------------------------------------------------------
+template <bool SR>
+__global__ void __launch_bounds__(256) mxfp8_cols_kernel(
+    const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
+    uint64_t offset, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int layout) {
+    __shared__ __align__(16) uint16_t tile[128][64 + 8];
+    const int64_t row_tiles = (rows + 127) / 128;
+    const int64_t col_tiles = cols / 64;
+    for (int64_t t = blockIdx.x; t < row_tiles * col_tiles; t += gridDim.x) {
+        const int64_t r0 = (t / col_tiles) * 128, c0 = (t % col_tiles) * 64;
+        const int nr = (int)(rows - r0 < 128 ? rows - r0 : 128);
+        __syncthreads();
+        for (int v = threadIdx.x; v < 128 * 8; v += 256) {
+            int rr = v >> 3, cc = (v & 7) * 8;
+            uint4 q = rr < nr ? __ldg(reinterpret_cast<const uint4 *>(x + (r0 + rr) * ld + c0 + cc))
+                              : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(&tile[rr][cc]) = q;
+        }
+        __syncthreads();
+        const int col = threadIdx.x & 63, rb = threadIdx.x >> 6;
+        if (rb * 32 < nr) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float((uint32_t)tile[rb * 32 + i][col] << 16);
+            float amax_b = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+            int k = mx_scale_exp(amax_b);
+            const int64_t c = c0 + col, rbase = r0 + rb * 32;
+            uint32_t w[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = 4 * q + j;
+                    uint32_t code;
+                    if (SR) {
+                        uint64_t idx = (uint64_t)((rbase + i) * cols + c);
+                        u32x4 r4 = philox_block(seed, offset, idx >> 2);
+                        uint32_t sel = (uint32_t)(idx & 3);
+                        uint32_t rw = sel == 0 ? r4.x : sel == 1 ? r4.y : sel == 2 ? r4.z : r4.w;
+                        code = e4m3_encode_sr(scale_pow2(v[i], k), rw);
+                    } else {
+                        code = e4m3_encode(scale_pow2(v[i], k));
+                    }
+                    word |= code << (8 * j);
+                }
+                w[q] = word;
+            }
+            uint4 *co = reinterpret_cast<uint4 *>(codes + c * rows + rbase);
+            co[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            co[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            const int64_t G = rows / 32;
+            const int64_t b = rbase / 32;
+            if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
+                scales[c * G + b] = (uint8_t)(k + 127);
+            else
+                scales[mma_sf_offset(c, b, G)] = (uint8_t)(k + 127);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) mxfp8_dequant_kernel(
+    const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales, int64_t n_rows,
+    int64_t n_cols, int layout, float *__restrict__ out) {
+    const int64_t G = n_cols / 32;
+    const int64_t n = n_rows * G;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, b = i - r * G;
+        uint32_t sc = layout == NVFP4MOE_LAYOUT_ROWMAJOR ? scales[r * G + b]
+                                                         : scales[mma_sf_offset(r, b, G)];
+        int k = (int)sc - 127;
+        const uint8_t *cp = codes + r * n_cols + b * 32;
+        float *op = out + r * n_cols + b * 32;
+        for (int j = 0; j < 32; ++j) op[j] = scale_pow2(e4m3_decode(cp[j]), -k);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// RHT32: per 32-element block, sign flip, five butterfly stages (h = 1, 2, 4,
+// 8, 16), times fp32(1/sqrt(32)); all in fp32 with one rounding per op.
+// ---------------------------------------------------------------------------
+NV_DEV void fwht32(float (&t)[32]) {
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if ((j & h) == 0) {
+                float a = t[j], b = t[j + h];
+                t[j] = __fadd_rn(a, b);
+                t[j + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+}
+
+#define RHT_C 0.17677669529663688f  // fp32 nearest to 1/sqrt(32)
+
+NV_DEV void rht32_fwd(const uint16_t *__restrict__ p, uint32_t signs, float (&v)[32]) {
+    const uint4 *pv = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) unpack8(__ldg(pv + j), v + 8 * j);
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        if ((signs >> i) & 1u) v[i] = -v[i];
+    fwht32(v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], RHT_C);
+}
+
+NV_DEV uint32_t rht_signs_dev(uint64_t sign_seed) {
+    return philox4x32_10(u32x4{0, 0, 0, 0}, (uint32_t)sign_seed, (uint32_t)(sign_seed >> 32)).x;
+}
+
+__global__ void __launch_bounds__(256) rht32_amax_kernel(const uint16_t *__restrict__ x,
+                                                         int64_t rows, int64_t cols, int64_t ld,
+                                                         uint64_t sign_seed,
+                                                         float *__restrict__ amax) {
+    const uint32_t signs = rht_signs_dev(sign_seed);
+    const int64_t G = cols / 32;
+    float m = 0.0f;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, b = i - r * G;
+        float v[32];
+        rht32_fwd(x + r * ld + b * 32, signs, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
+    m = warp_max(m);
+    __shared__ float red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+        v = warp_max(v);
+        if (threadIdx.x == 0) atomic_max_nonneg(amax, v);
+    }
+}
+
+__global__ void __launch_bounds__(256) rht32_quant_kernel(
+    const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t sign_seed,
+    int fmt, const float *__restrict__ amax_p, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ scales, float *__restrict__ ts_out) {
+    const uint32_t signs = rht_signs_dev(sign_seed);
+    const int64_t G = cols / 32;
+    float S_enc = 1.0f;
+    if (fmt == NVFP4MOE_FMT_NVFP4) {
+        float amax = *amax_p;
+        S_enc = nvfp4_senc(amax);
+        if (ts_out && blockIdx.x == 0 && threadIdx.x == 0) *ts_out = nvfp4_ts(amax);
+    }
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, b = i - r * G;
+        float v[32];
+        rht32_fwd(x + r * ld + b * 32, signs, v);
+        if (fmt == NVFP4MOE_FMT_NVFP4) {
+            float h0[16], h1[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) { h0[j] = v[j]; h1[j] = v[16 + j]; }
+            uint32_t w0, w1, w2, w3;
+            uint32_t s0 = nvfp4_block16(h0, S_enc, w0, w1);
+            uint32_t s1 = nvfp4_block16(h1, S_enc, w2, w3);
+            *reinterpret_cast<uint4 *>(codes + r * (cols / 2) + b * 16) = make_uint4(w0, w1, w2, w3);
+            *reinterpret_cast<uint16_t *>(scales + r * (cols / 16) + b * 2) =
+                (uint16_t)(s0 | (s1 << 8));
+        } else {
+            uint32_t w[8];
+            uint32_t sc = mx_block32<false>(v, 0, 0, 0, w);
+            uint4 *co = reinterpret_cast<uint4 *>(codes + r * cols + b * 32);
+            co[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            co[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            scales[r * G + b] = (uint8_t)sc;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) rht32_dequant_kernel(
+    const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+    const float *__restrict__ ts_p, int64_t rows, int64_t cols, uint64_t sign_seed, int fmt,
+    float *__restrict__ out) {
+    const uint32_t signs = rht_signs_dev(sign_seed);
+    const int64_t G = cols / 32;
+    const float ts = (fmt == NVFP4MOE_FMT_NVFP4) ? *ts_p : 1.0f;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, b = i - r * G;
+        float t[32];
+        if (fmt == NVFP4MOE_FMT_NVFP4) {
+            uint4 q = *reinterpret_cast<const uint4 *>(codes + r * (cols / 2) + b * 16);
+            uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+            float sf0 = e4m3_decode(scales[r * (cols / 16) + 2 * b]);
+            float sf1 = e4m3_decode(scales[r * (cols / 16) + 2 * b + 1]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                float sf = j < 16 ? sf0 : sf1;
+                t[j] = __fmul_rn(e2m1_decode((qs[j >> 3] >> (4 * (j & 7))) & 15u) * sf, ts);
+            }
+        } else {
+            int k = (int)scales[r * G + b] - 127;
+            const uint4 *cq = reinterpret_cast<const uint4 *>(codes + r * cols + b * 32);
+            uint4 q0 = cq[0], q1 = cq[1];
+            uint32_t qs[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                t[j] = scale_pow2(e4m3_decode((qs[j >> 2] >> (8 * (j & 3))) & 0xFFu), -k);
+        }
+        fwht32(t);
+        float *op = out + r * cols + b * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            float u = __fmul_rn(t[j], RHT_C);
+            t[j] = ((signs >> j) & 1u) ? -u : u;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4 *>(op + j) = make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+static int grid_for(int64_t work, int per_block = 256) {
+    int64_t g = (work + per_block - 1) / per_block;
+    const int64_t cap = 148 * 16;
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return (int)g;
+}
+
+cudaError_t launch_amax_bf16(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                             float *amax, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    if (rows * cols == 0) return cudaSuccess;
+    amax_bf16_kernel<<<grid_for(rows * (cols / 8)), 256, 0, s>>>(x, rows, cols, ld, amax);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                  const float *amax_in, uint8_t *codes, uint8_t *scales,
+                                  float *ts_out, int layout, cudaStream_t s) {
+    cudaError_t e;
+    if (!amax_in) {
+        // ts_out holds the amax between the passes, then becomes amax / 2688
+        if ((e = launch_amax_bf16(x, rows, cols, ld, ts_out, s)) != cudaSuccess) return e;
+        if (rows * cols > 0)
+            nvfp4_quant_kernel<<<grid_for(rows * (cols / 64)), 256, 0, s>>>(
+                x, rows, cols, ld, ts_out, codes, scales, nullptr, layout);
+        nvfp4_finalize_ts_kernel<<<1, 1, 0, s>>>(ts_out);
+    } else {
+        nvfp4_quant_kernel<<<grid_for(rows * (cols / 64)), 256, 0, s>>>(
+            x, rows, cols, ld, amax_in, codes, scales, ts_out, layout);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                    int64_t rows, int64_t cols, int layout, float *out,
+                                    cudaStream_t s) {
+    if (rows * cols == 0) return cudaSuccess;
+    nvfp4_dequant_kernel<<<grid_for(rows * (cols / 16)), 256, 0, s>>>(codes, scales, ts, rows,
+                                                                      cols, layout, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp8_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                  int axis, uint64_t seed, uint64_t offset, int rounding,
+                                  uint8_t *codes, uint8_t *scales, int layout, cudaStream_t s) {
+    if (rows * cols == 0) return cudaSuccess;
+    const bool sr = rounding == NVFP4MOE_ROUND_SR;
+    if (axis == 0) {
+        int g = grid_for(rows * (cols / 32));
+        if (sr)
+            mxfp8_rows_kernel<true><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes, scales,
+                                                      layout);
+        else
+            mxfp8_rows_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes,
+                                                       scales, layout);
+    } else {
+        int64_t tiles = ((rows + 127) / 128) * (cols / 64);
+        int g = (int)(tiles < 148 * 8 ? tiles : 148 * 8);
+        if (sr)
+            mxfp8_cols_kernel<true><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes, scales,
+                                                      layout);
+        else
+            mxfp8_cols_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes,
+                                                       scales, layout);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp8_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t n_rows,
+                                    int64_t n_cols, int layout, float *out, cudaStream_t s) {
+    if (n_rows * n_cols == 0) return cudaSuccess;
+    mxfp8_dequant_kernel<<<grid_for(n_rows * (n_cols / 32)), 256, 0, s>>>(codes, scales, n_rows,
+                                                                          n_cols, layout, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rht32_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                  uint64_t sign_seed, int fmt, const float *amax_in,
+                                  uint8_t *codes, uint8_t *scales, float *ts_out,
+                                  cudaStream_t s) {
+    cudaError_t e;
+    const int g = grid_for(rows * (cols / 32));
+    if (fmt == NVFP4MOE_FMT_NVFP4 && !amax_in) {
+        if ((e = cudaMemsetAsync(ts_out, 0, sizeof(float), s)) != cudaSuccess) return e;
+        if (rows * cols > 0) {
+            rht32_amax_kernel<<<g, 256, 0, s>>>(x, rows, cols, ld, sign_seed, ts_out);
+            rht32_quant_kernel<<<g, 256, 0, s>>>(x, rows, cols, ld, sign_seed, fmt, ts_out, codes,
+                                                 scales, nullptr);
+        }
+        nvfp4_finalize_ts_kernel<<<1, 1, 0, s>>>(ts_out);
+    } else if (rows * cols > 0) {
+        rht32_quant_kernel<<<g, 256, 0, s>>>(x, rows, cols, ld, sign_seed, fmt, amax_in, codes,
+                                             scales, ts_out);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rht32_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                    int64_t rows, int64_t cols, uint64_t sign_seed, int fmt,
+                                    float *out, cudaStream_t s) {
+    if (rows * cols == 0) return cudaSuccess;
+    rht32_dequant_kernel<<<grid_for(rows * (cols / 32)), 256, 0, s>>>(codes, scales, ts, rows, cols,
+                                                                      sign_seed, fmt, out);
+    return cudaGetLastError();
+}
+
+// grouped NVFP4 quantization of the expert activations h with per-expert
+// tensor scales: rows [off[e], off[e+1]) use amax[e]; ts[e] = amax[e] / 2688.
+__global__ void __launch_bounds__(256) nvfp4_quant_grouped_kernel(
+    const uint16_t *__restrict__ x, int64_t cols, const int32_t *__restrict__ off, int32_t E,
+    const float *__restrict__ amax, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+    float *__restrict__ ts) {
+    extern __shared__ int32_t s_off[];
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = off[i];
+    __syncthreads();
+    if (blockIdx.x == 0)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) ts[e] = nvfp4_ts(amax[e]);
+    const int64_t rows = s_off[E];
+    const int64_t G = cols / 64;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t r = i / G, g = i - r * G;
+        int lo = 0, hi = E;  // largest e with s_off[e] <= r
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (s_off[mid] <= r) lo = mid; else hi = mid;
+        }
+        const float S_enc = nvfp4_senc(amax[lo]);
+        uint4 c0, c1;
+        uint32_t scw = nvfp4_quant64(x + r * cols + g * 64, S_enc, c0, c1);
+        uint4 *co = reinterpret_cast<uint4 *>(codes + r * (cols / 2) + g * 32);
+        co[0] = c0;
+        co[1] = c1;
+        *reinterpret_cast<uint32_t *>(scales + mma_sf_offset(r, g * 4, cols / 16)) = scw;
+    }
+}
+
+cudaError_t launch_nvfp4_quant_grouped(const uint16_t *x, int64_t rows_alloc, int64_t cols,
+                                       const int32_t *off, int32_t E, const float *amax,
+                                       uint8_t *codes, uint8_t *scales, float *ts,
+                                       cudaStream_t s) {
+    int g = grid_for(rows_alloc * (cols / 64));
+    nvfp4_quant_grouped_kernel<<<g, 256, (E + 1) * sizeof(int32_t), s>>>(x, cols, off, E, amax,
+                                                                         codes, scales, ts);
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4moe

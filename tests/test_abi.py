@@ -1,0 +1,89 @@
+"""The C ABI library loads without a GPU, exports every entry point the header
+declares, and rejects bad arguments on the host before launching anything."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from precision_moe_numerics_quantize_b200 import build as B
+from precision_moe_numerics_quantize_b200 import nvfp4moe as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return M.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_0-9]+)\s*\(", src,
+                       flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["nvfp4_quantize", "mxfp8_quantize_sr", "rht32_quantize", "moe_route_permute",
+              "moe_expert_fwd", "moe_combine", "nvfp4_grouped_gemm", "mxfp8_grouped_gemm"]:
+        assert n in names
+    assert set(names) == set(M.EXPORTED), set(names) ^ set(M.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_host_only_queries(L):
+    assert L.nvfp4moe_version() == 100
+    assert L.nvfp4moe_max_rows(16384, 8, 384) == (16384 * 8 + 384 * 127 + 127) // 128 * 128
+    assert L.nvfp4moe_max_rows(0, 1, 1) == 128
+    assert L.moe_route_permute_workspace_size(16384, 384, 8) > 0
+    assert L.moe_route_permute_workspace_size(10, 0, 1) == 0
+
+
+P = 1 << 20  # a fake, 16-byte aligned "device pointer"; validation fails before any use
+
+
+@pytest.mark.parametrize("call,status", [
+    (lambda L: L.nvfp4_quantize(P, 4, 48, 48, None, P, P, P + 16, 0, None), 2),      # cols % 64
+    (lambda L: L.nvfp4_quantize(P, 100, 64, 64, None, P, P, P + 16, 1, None), 2),    # MMA rows
+    (lambda L: L.nvfp4_quantize(P + 2, 4, 64, 64, None, P, P, P + 16, 0, None), 3),  # align
+    (lambda L: L.nvfp4_quantize(None, 4, 64, 64, None, P, P, P + 16, 0, None), 1),   # null
+    (lambda L: L.nvfp4_quantize(P, 4, 64, 64, P + 16, P, P, P + 16, 0, None), 1),    # alias
+    (lambda L: L.nvfp4_quantize(P, 4, 64, 64, None, P, P, P + 16, 7, None), 1),      # layout
+    (lambda L: L.mxfp8_quantize_sr(P, 4, 64, 64, 2, 0, 0, 1, P, P, 0, None), 1),     # axis
+    (lambda L: L.mxfp8_quantize_sr(P, 40, 64, 64, 1, 0, 0, 1, P, P, 0, None), 2),    # rows % 32
+    (lambda L: L.mxfp8_quantize_sr(P, 4, 64, 64, 0, 0, 0, 5, P, P, 0, None), 1),     # rounding
+    (lambda L: L.rht32_quantize(P, 4, 48, 48, 0, 0, None, P, P, P, 0, None), 2),     # cols % 32
+    (lambda L: L.rht32_quantize(P, 4, 64, 64, 0, 0, None, P, P, P, 1, None), 7),     # MMA layout
+    (lambda L: L.moe_route_permute(P, P, 8, 4, 5, 64, 1, None, P, P, P, P, P, P, P, P, P,
+                                   1 << 20, None), 1),                               # k > E
+    (lambda L: L.moe_route_permute(P, P, 8, 4, 2, 64, 1, None, P, P, P, P, P, P, P, P, P,
+                                   4, None), 4),                                     # workspace
+    (lambda L: L.moe_route_permute(P, P, 8, 4, 2, 96, 1, None, P, P, P, P, P, P, P, P, P,
+                                   1 << 20, None), 2),                               # d % 64
+    (lambda L: L.moe_expert_fwd(P, P, P, P, 4, 384, 256, P, P, P, P, P, P, P, P, P, P, P, P,
+                                128, None), 2),                                      # d % 256
+    (lambda L: L.moe_combine(P, P, P, 4, 2, 12, P, None), 2),                        # d % 8
+    (lambda L: L.nvfp4_grouped_gemm(P, P, P, 2, P, P, P, P, 1, 128, 256, 256, P, 0, None), 1),
+    (lambda L: L.nvfp4_grouped_gemm(P, P, P, 0, P, P, P, P, 1, 128, 256, 128, P, 0, None), 2),
+    (lambda L: L.mxfp8_grouped_gemm(P, P, P, P, P, 1, 3, 128, 256, 128, P, 1, None), 1),
+    (lambda L: L.mxfp8_grouped_gemm(P, P, P, P, P, 2000, 0, 128, 256, 128, P, 1, None), 1),
+])
+def test_validation_rejects_before_launch(L, call, status):
+    assert call(L) == status
+    assert L.nvfp4moe_last_error().decode()
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        M.nvfp4_quantize(x, x, x, x)
