@@ -69,7 +69,7 @@ class ClockSampler:
             uuid = "GPU-" + str(torch.cuda.get_device_properties(dev_index).uuid)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -376,6 +376,21 @@ def run_reference(args, shape):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(x, dist, device):
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def replica_value(flops_per_step, ms_per_step, world):
+    """Whole-job TFLOPS of `world` replicas timed by the slowest rank."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 def workload_name(args, shape):
     return (f"{args.workload} router={args.router}: T={shape.T} d={shape.d} f={shape.f} "
             f"E={shape.E} top-{shape.k} SwiGLU")
@@ -388,7 +403,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["full_moe", "small_moe"], default="full_moe")
+    ap.add_argument("--workload", choices=["full_moe", "small_moe", "mid_moe"], default="full_moe")
     ap.add_argument("--router", choices=["uniform", "zipf"], default="uniform")
     ap.add_argument("--no-companions", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -433,19 +448,17 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    # the profiler window covers exactly the timed steps (ncu --profile-from-start off)
+    torch.cuda.profiler.start()
     total_ms, per_call = time_calls(torch, calls, args.steps)
     torch.cuda.synchronize()
+    torch.cuda.profiler.stop()
     if dist:
         dist.barrier()
-    clocks = sampler.stop()
-    ms = total_ms / args.steps
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks(total_ms / args.steps, dist, dev)
     T, d, f, E, k = shape.T, shape.d, shape.f, shape.E, shape.k
     flops = 6.0 * T * k * d * f
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = replica_value(flops, ms, world)
 
     # ---- end to end: host buffers, copies inside the timed region ----
     stream = torch.cuda.current_stream()
@@ -463,12 +476,9 @@ def main():
         L["out_host"].copy_(L["out"], non_blocking=True)
     eb.record()
     torch.cuda.synchronize()
-    e2e_ms = ea.elapsed_time(eb) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+    clocks = sampler.stop()
+    e2e_ms = max_over_ranks(ea.elapsed_time(eb) / args.steps, dist, dev)
+    e2e = {"value": replica_value(flops, e2e_ms, world), "unit": "TFLOPS",
            "h2d_bytes_per_step": L["x_host"].numel() * 2 + L["logits_host"].numel() * 4,
            "d2h_bytes_per_step": L["out_host"].numel() * 2, "ms_per_step": e2e_ms}
     del stream

@@ -167,6 +167,8 @@ class MoEShape:
 SHAPES = {
     "single_gemm": None,  # A [128 x 256], W [256 x 256]
     "small_moe": MoEShape(T=2048, d=1024, f=512, E=32, k=4),
+    # profiling case: full hidden sizes, 64 experts (1.1 GB of NVFP4 weights)
+    "mid_moe": MoEShape(T=4096, d=4096, f=2560, E=64, k=8),
     "full_moe": MoEShape(T=16384, d=4096, f=2560, E=384, k=8),
 }
 
