@@ -207,6 +207,30 @@ nvfp4moe_status moe_route_permute(const float *logits, const uint16_t *x, int64_
                                   float *x_ts, void *ws, size_t ws_bytes,
                                   nvfp4moe_stream_t stream);
 
+/* The same routing and dispatch without a workspace argument. The pages have
+ * no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory: a process whose device memory is reserved up front
+ * by another runtime's allocator (a serving engine holding almost all HBM),
+ * so that a cudaMalloc would fail; code called from inside another framework
+ * that must not allocate on its own; and latency-critical loops that cannot
+ * afford cudaMalloc's implicit device synchronisation.
+ * The scratch is a 4 MiB array inside the library (held by every GPU that
+ * loads the library until the process exits); calls needing more, i.e. when
+ * moe_route_permute_workspace_size(T, E, k) > 4 MiB, are rejected with
+ * NVFP4MOE_ERR_WORKSPACE before anything is launched. The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and
+ * caches it; make that first call before any stream capture. Every call on a
+ * device uses the same array and the kernels overwrite all of it that they
+ * read, so nothing needs clearing between calls, but two calls that overlap
+ * on the GPU (different streams, no ordering between them) race on it.
+ * Arguments, outputs and errors are otherwise those of moe_route_permute. */
+nvfp4moe_status moe_route_permute_noalloc(const float *logits, const uint16_t *x, int64_t T,
+                                          int32_t E, int32_t k, int64_t d, int renorm,
+                                          const float *x_amax_in, int32_t *topk_idx,
+                                          float *topk_w, int32_t *expert_off, int32_t *pos,
+                                          int32_t *token_of, uint8_t *xq, uint8_t *xq_sc,
+                                          float *x_ts, nvfp4moe_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Expert FFN forward in NVFP4 (news.t0001.com '训练数值格式分工清单'; aicoder.com
  * 'Architecture highlights': NVFP4 forward in the expert layers).

@@ -74,6 +74,42 @@ static nvfp4moe_status after_launch(cudaError_t e, const char *what) {
     return cuda_status(e, what);
 }
 
+namespace nvfp4moe {
+
+// Argument checks shared by the entry points that route and dispatch.
+nvfp4moe_status check_route_permute_args(const float *logits, const uint16_t *x, int64_t T,
+                                         int32_t E, int32_t k, int64_t d, int renorm,
+                                         const float *x_amax_in, const int32_t *topk_idx,
+                                         const float *topk_w, const int32_t *expert_off,
+                                         const int32_t *pos, const int32_t *token_of,
+                                         const uint8_t *xq, const uint8_t *xq_sc,
+                                         const float *x_ts) {
+    NEED(T >= 0 && d > 0, NVFP4MOE_ERR_INVALID_ARG, "moe_route_permute: T >= 0 and d > 0 required");
+    NEED(E >= 1 && E <= 1024, NVFP4MOE_ERR_INVALID_ARG, "moe_route_permute: 1 <= E <= 1024");
+    NEED(k >= 1 && k <= 32 && k <= E, NVFP4MOE_ERR_INVALID_ARG,
+         "moe_route_permute: 1 <= k <= min(E, 32) required (k=%d, E=%d)", k, E);
+    NEED(renorm == 0 || renorm == 1, NVFP4MOE_ERR_INVALID_ARG, "moe_route_permute: renorm 0 or 1");
+    NEED(d % 64 == 0, NVFP4MOE_ERR_SHAPE, "moe_route_permute: d %% 64 == 0 required");
+    NEED(T * k <= 0x7FFFFFFFLL - (int64_t)E * 128, NVFP4MOE_ERR_SHAPE,
+         "moe_route_permute: T*k too large for int32 row indices");
+    NEED_PTR4(expert_off);
+    NEED_PTR4(token_of);
+    NEED_PTR4(x_ts);
+    NEED_PTR(xq);
+    NEED_PTR(xq_sc);
+    if (T > 0) {
+        NEED_PTR4(logits);
+        NEED_PTR(x);
+        NEED_PTR4(topk_idx);
+        NEED_PTR4(topk_w);
+        NEED_PTR4(pos);
+    }
+    OPT_PTR4(x_amax_in);
+    return NVFP4MOE_OK;
+}
+
+}  // namespace nvfp4moe
+
 extern "C" {
 
 int nvfp4moe_version(void) { return 100; }
@@ -261,27 +297,10 @@ nvfp4moe_status moe_route_permute(const float *logits, const uint16_t *x, int64_
                                   int32_t *pos, int32_t *token_of, uint8_t *xq, uint8_t *xq_sc,
                                   float *x_ts, void *ws, size_t ws_bytes,
                                   nvfp4moe_stream_t stream) {
-    NEED(T >= 0 && d > 0, NVFP4MOE_ERR_INVALID_ARG, "moe_route_permute: T >= 0 and d > 0 required");
-    NEED(E >= 1 && E <= 1024, NVFP4MOE_ERR_INVALID_ARG, "moe_route_permute: 1 <= E <= 1024");
-    NEED(k >= 1 && k <= 32 && k <= E, NVFP4MOE_ERR_INVALID_ARG,
-         "moe_route_permute: 1 <= k <= min(E, 32) required (k=%d, E=%d)", k, E);
-    NEED(renorm == 0 || renorm == 1, NVFP4MOE_ERR_INVALID_ARG, "moe_route_permute: renorm 0 or 1");
-    NEED(d % 64 == 0, NVFP4MOE_ERR_SHAPE, "moe_route_permute: d %% 64 == 0 required");
-    NEED(T * k <= 0x7FFFFFFFLL - (int64_t)E * 128, NVFP4MOE_ERR_SHAPE,
-         "moe_route_permute: T*k too large for int32 row indices");
-    NEED_PTR4(expert_off);
-    NEED_PTR4(token_of);
-    NEED_PTR4(x_ts);
-    NEED_PTR(xq);
-    NEED_PTR(xq_sc);
-    if (T > 0) {
-        NEED_PTR(logits);
-        NEED_PTR(x);
-        NEED_PTR4(topk_idx);
-        NEED_PTR4(topk_w);
-        NEED_PTR4(pos);
-    }
-    OPT_PTR4(x_amax_in);
+    nvfp4moe_status st = check_route_permute_args(logits, x, T, E, k, d, renorm, x_amax_in,
+                                                  topk_idx, topk_w, expert_off, pos, token_of,
+                                                  xq, xq_sc, x_ts);
+    if (st) return st;
     NEED(ws != nullptr && ws_bytes >= route_permute_ws_bytes(T, E, k), NVFP4MOE_ERR_WORKSPACE,
          "moe_route_permute: workspace of %zu bytes needed", route_permute_ws_bytes(T, E, k));
     NEED(aligned16(ws), NVFP4MOE_ERR_ALIGN, "moe_route_permute: ws is not 16-byte aligned");

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/nvfp4moe.h"
+
 namespace nvfp4moe {
 
 cudaError_t launch_amax_bf16(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
@@ -37,6 +39,13 @@ cudaError_t launch_route_permute(const float *logits, const uint16_t *x, int64_t
                                  int32_t *topk_idx, float *topk_w, int32_t *expert_off,
                                  int32_t *pos, int32_t *token_of, uint8_t *xq, uint8_t *xq_sc,
                                  float *x_ts, void *ws, int64_t rows_alloc, cudaStream_t s);
+nvfp4moe_status check_route_permute_args(const float *logits, const uint16_t *x, int64_t T,
+                                         int32_t E, int32_t k, int64_t d, int renorm,
+                                         const float *x_amax_in, const int32_t *topk_idx,
+                                         const float *topk_w, const int32_t *expert_off,
+                                         const int32_t *pos, const int32_t *token_of,
+                                         const uint8_t *xq, const uint8_t *xq_sc,
+                                         const float *x_ts);
 cudaError_t launch_combine(const uint16_t *y, const int32_t *pos, const float *w, int64_t T,
                            int32_t k, int64_t d, uint16_t *out, cudaStream_t s);
 

@@ -391,3 +391,76 @@ cudaError_t launch_combine(const uint16_t *y, const int32_t *pos, const float *w
 }
 
 }  // namespace nvfp4moe
+
+// ---------------------------------------------------------------------------
+// Dispatch without a caller-provided workspace: the scratch lives in a
+// file-scope device array of fixed size, shared by every call on a device.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace nvfp4moe {
+
+static constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+
+// Every GPU that loads the library keeps this array until the process exits.
+static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocScratchBytes];
+
+// Device address of g_route_scratch on the current device. In host code the
+// array's name is only a stand-in, so the address is looked up once per
+// device with cudaGetSymbolAddress (the first call on a device) and cached.
+static void *route_scratch_address(nvfp4moe_status *st) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        *st = cuda_status(e, "moe_route_permute_noalloc: cudaGetDevice");
+        return nullptr;
+    }
+    if (dev < 0 || dev >= kMaxDevices) {
+        set_last_error("moe_route_permute_noalloc: device %d out of range", dev);
+        *st = NVFP4MOE_ERR_INVALID_ARG;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess) {
+            *st = cuda_status(e, "moe_route_permute_noalloc: cudaGetSymbolAddress");
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace nvfp4moe
+
+extern "C" nvfp4moe_status moe_route_permute_noalloc(
+    const float *logits, const uint16_t *x, int64_t T, int32_t E, int32_t k, int64_t d,
+    int renorm, const float *x_amax_in, int32_t *topk_idx, float *topk_w, int32_t *expert_off,
+    int32_t *pos, int32_t *token_of, uint8_t *xq, uint8_t *xq_sc, float *x_ts,
+    nvfp4moe_stream_t stream) {
+    using namespace nvfp4moe;
+    nvfp4moe_status st = check_route_permute_args(logits, x, T, E, k, d, renorm, x_amax_in,
+                                                  topk_idx, topk_w, expert_off, pos, token_of,
+                                                  xq, xq_sc, x_ts);
+    if (st) return st;
+    const size_t need = route_permute_ws_bytes(T, E, k);
+    if (need > kNoAllocScratchBytes) {
+        set_last_error(
+            "moe_route_permute_noalloc: T=%lld, E=%d, k=%d needs %zu bytes of scratch, more than "
+            "the built-in %zu; use moe_route_permute with a workspace",
+            (long long)T, E, k, need, kNoAllocScratchBytes);
+        return NVFP4MOE_ERR_WORKSPACE;
+    }
+    void *ws = route_scratch_address(&st);
+    if (!ws) return st;
+    cudaError_t e = launch_route_permute(logits, x, T, E, k, d, renorm, x_amax_in, topk_idx,
+                                         topk_w, expert_off, pos, token_of, xq, xq_sc, x_ts, ws,
+                                         nvfp4moe_max_rows(T, k, E), (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return cuda_status(e, "moe_route_permute_noalloc");
+}

@@ -52,6 +52,8 @@ _SIGS = {
     "moe_route_permute_workspace_size": (_SZ, [_I64, _I32, _I32]),
     "moe_route_permute": (C.c_int, [_P, _P, _I64, _I32, _I32, _I64, _I, _P, _P, _P, _P, _P, _P,
                                     _P, _P, _P, _P, _SZ, _P]),
+    "moe_route_permute_noalloc": (C.c_int, [_P, _P, _I64, _I32, _I32, _I64, _I, _P, _P, _P, _P,
+                                            _P, _P, _P, _P, _P, _P]),
     "moe_expert_fwd": (C.c_int, [_P, _P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                  _P, _P, _P, _P, _P, _I64, _P]),
     "moe_combine": (C.c_int, [_P, _P, _P, _I64, _I32, _I64, _P, _P]),
@@ -177,6 +179,17 @@ def moe_route_permute(logits, x, k, renorm, topk_idx, topk_w, expert_off, pos, t
         _ptr(logits), _ptr(x), T, E, k, d, renorm, _ptr(x_amax_in), _ptr(topk_idx), _ptr(topk_w),
         _ptr(expert_off), _ptr(pos), _ptr(token_of), _ptr(xq), _ptr(xq_sc), _ptr(x_ts), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_route_permute_noalloc(logits, x, k, renorm, topk_idx, topk_w, expert_off, pos, token_of,
+                              xq, xq_sc, x_ts, x_amax_in=None, stream=None):
+    """moe_route_permute with the library's built-in scratch instead of a workspace."""
+    T, E = logits.shape
+    d = x.shape[1]
+    _check("moe_route_permute_noalloc", lib().moe_route_permute_noalloc(
+        _ptr(logits), _ptr(x), T, E, k, d, renorm, _ptr(x_amax_in), _ptr(topk_idx), _ptr(topk_w),
+        _ptr(expert_off), _ptr(pos), _ptr(token_of), _ptr(xq), _ptr(xq_sc), _ptr(x_ts),
+        _stream(stream)))
 
 
 def moe_expert_fwd(xq, xq_sc, x_ts, expert_off, E, d, f, w1, w1_sc, w1_ts, w2, w2_sc, w2_ts, h,
