@@ -104,6 +104,15 @@ const char *nvfp4moe_last_error(void);
  * identifier of the wait that ran out. Returns NVFP4MOE_ERR_TIMEOUT if set. */
 nvfp4moe_status nvfp4moe_device_error(int32_t *code);
 
+/* Exhaustive check of the hardware conversions the quantizers use against the
+ * library's own encoders (which the test suite pins bit for bit to the CPU
+ * reference): which = 0 checks cvt.rn.satfinite.e2m1x2.f32, which = 1
+ * cvt.rn.satfinite.e4m3x2.f32, each over every finite fp32 input. The
+ * mismatch count lands in *mismatches (device uint64, overwritten). Has no
+ * counterpart on the pages; it guards the encoders on a new driver. */
+nvfp4moe_status nvfp4moe_selftest(int which, unsigned long long *mismatches,
+                                  nvfp4moe_stream_t stream);
+
 /* Upper bound on the rows of a permuted, per-expert-padded activation:
  * T*k + E*127 rounded up to 128. Pure host arithmetic. */
 int64_t nvfp4moe_max_rows(int64_t T, int32_t k, int32_t E);

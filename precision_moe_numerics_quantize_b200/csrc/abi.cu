@@ -129,6 +129,14 @@ nvfp4moe_status nvfp4moe_device_error(int32_t *code) {
     return NVFP4MOE_OK;
 }
 
+nvfp4moe_status nvfp4moe_selftest(int which, unsigned long long *mismatches,
+                                  nvfp4moe_stream_t stream) {
+    NEED(which == 0 || which == 1, NVFP4MOE_ERR_INVALID_ARG, "nvfp4moe_selftest: which is 0 or 1");
+    NEED_PTR4(mismatches);
+    return after_launch(launch_selftest(which, mismatches, (cudaStream_t)stream),
+                        "nvfp4moe_selftest");
+}
+
 int64_t nvfp4moe_max_rows(int64_t T, int32_t k, int32_t E) {
     if (T < 0 || k < 0 || E < 0) return 0;
     return (T * k + (int64_t)E * 127 + 127) / 128 * 128;

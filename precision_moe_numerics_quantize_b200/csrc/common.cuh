@@ -112,6 +112,33 @@ NV_DEV float e4m3_decode(uint32_t c) {
     return (c & 0x80u) ? -v : v;
 }
 
+// ---------------------------------------------------------------------------
+// Hardware conversions (sm_100a cvt.rn.satfinite). They round to nearest with
+// ties to even and saturate, as the encoders above do; nvfp4moe_selftest
+// compares them with those encoders over every finite fp32 input.
+// ---------------------------------------------------------------------------
+// Eight floats -> eight E2M1 codes in one word, v[0] in the lowest nibble.
+NV_DEV uint32_t e2m1x8_hw(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                          float v7) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return r;
+}
+
+// Two floats -> two E4M3 codes, lo in the low byte.
+NV_DEV uint32_t e4m3x2_hw(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // 2^e as an fp32 for e in [-126, 127].
 NV_DEV float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
 
@@ -157,6 +184,46 @@ NV_DEV uint32_t e4m3_encode_sr(float v, uint32_t r) {
 }
 
 // ---------------------------------------------------------------------------
+// NVFP4 block of 16: per-tensor S_enc, block scale s = E4M3((amax_b / 6) * S_enc),
+// codes E2M1(x * S_enc / s). Returns the scale code; 8 code bytes in w0, w1.
+// ---------------------------------------------------------------------------
+NV_DEV float nvfp4_senc(float amax) {
+    return (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(2688.0f, amax) : 1.0f;
+}
+NV_DEV float nvfp4_ts(float amax) {
+    return (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+NV_DEV uint32_t nvfp4_block16(const float *v, float S_enc, uint32_t &w0, uint32_t &w1) {
+    float amax_b = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+    const float t = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S_enc);
+    const uint32_t sc = e4m3_encode_pos(t);
+    const float sf = e4m3_decode_pos(sc);
+    const float enc = (sf == 0.0f) ? 0.0f : __fdiv_rn(S_enc, sf);
+    w0 = e2m1x8_hw(__fmul_rn(v[0], enc), __fmul_rn(v[1], enc), __fmul_rn(v[2], enc),
+                   __fmul_rn(v[3], enc), __fmul_rn(v[4], enc), __fmul_rn(v[5], enc),
+                   __fmul_rn(v[6], enc), __fmul_rn(v[7], enc));
+    w1 = e2m1x8_hw(__fmul_rn(v[8], enc), __fmul_rn(v[9], enc), __fmul_rn(v[10], enc),
+                   __fmul_rn(v[11], enc), __fmul_rn(v[12], enc), __fmul_rn(v[13], enc),
+                   __fmul_rn(v[14], enc), __fmul_rn(v[15], enc));
+    return sc;
+}
+
+NV_DEV void unpack_bf16x8(uint4 q, float *f) {
+    f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x); f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
+    f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z); f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
+}
+
+// Byte offset of scale (row r, scale column c) in the MMA layout of a matrix
+// whose rows carry nsc scales (nsc % 4 == 0).
+NV_DEV size_t mma_sf_offset(int64_t r, int64_t c, int64_t nsc) {
+    int64_t chunk = (r >> 7) * (nsc >> 2) + (c >> 2);
+    return (size_t)chunk * 512 + (size_t)((r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3));
+}
+
+// ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon et al., SC'11): 10 rounds of the multiply-xor bijection
 // with the published multipliers and Weyl key increments.
 // ---------------------------------------------------------------------------
@@ -165,9 +232,11 @@ struct u32x4 { uint32_t x, y, z, w; };
 NV_DEV u32x4 philox4x32_10(u32x4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
     for (int i = 0; i < 10; ++i) {
-        uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-        uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
-        c = u32x4{hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0};
+        // one 32x32 -> 64-bit multiply gives both halves of each product
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c.x;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c.z;
+        c = u32x4{(uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1,
+                  (uint32_t)p0};
         k0 += 0x9E3779B9u;
         k1 += 0xBB67AE85u;
     }

@@ -344,24 +344,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_after();
             }
             const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+            // Drain this warp's 128 accumulator columns into registers, hand the
+            // accumulator back to the MMA warp at once, then do the math and the
+            // stores while the next tile's MMAs run.
+            uint32_t acc[4][32];
+            if (have_acc) {
+                if (p.epi == EPI_SWIGLU_AMAX) {
+                    tmem_ld_32x32b_x32(lane_addr + half * 64, acc[0]);           // gate
+                    tmem_ld_32x32b_x32(lane_addr + half * 64 + 32, acc[1]);
+                    tmem_ld_32x32b_x32(lane_addr + 128 + half * 64, acc[2]);     // up
+                    tmem_ld_32x32b_x32(lane_addr + 128 + half * 64 + 32, acc[3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        tmem_ld_32x32b_x32(lane_addr + half * 128 + c * 32, acc[c]);
+                }
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[c][i] = 0u;
+            }
             if (p.epi == EPI_SWIGLU_AMAX) {
                 uint16_t *h = static_cast<uint16_t *>(p.c);
                 float amax = 0.0f;
-#pragma unroll 1
+#pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int hc = half * 64 + c * 32;
-                    uint32_t gr[32], ur[32];
-                    tmem_ld_32x32b_x32(lane_addr + hc, gr);
-                    tmem_ld_32x32b_x32(lane_addr + 128 + hc, ur);
-                    tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         float hv[2];
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            const float gq = __fmul_rn(__uint_as_float(gr[i + j]), alpha);
-                            const float uq = __fmul_rn(__uint_as_float(ur[i + j]), alpha);
+                            const float gq = __fmul_rn(__uint_as_float(acc[c][i + j]), alpha);
+                            const float uq = __fmul_rn(__uint_as_float(acc[2 + c][i + j]), alpha);
                             const float den = fminf(1.0f + __expf(-gq), 1e30f);
                             hv[j] = __fmul_rn(__fdividef(gq, den), uq);
                         }
@@ -375,31 +396,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int v = 0; v < 4; ++v)
                         dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
                 amax = warp_max(amax);
                 if (lane == 0) atomic_max_nonneg(p.amax + T.g, amax);
             } else {
-#pragma unroll 1
+#pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int col = half * 128 + c * 32;
-                    uint32_t r[32];
-                    if (have_acc) {
-                        tmem_ld_32x32b_x32(lane_addr + col, r);
-                        tmem_wait_ld();
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = 0u;
-                    }
                     if (p.epi == EPI_STORE_BF16) {
                         uint16_t *cp = static_cast<uint16_t *>(p.c) + row * p.ldc + T.out_col + col;
                         uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 32; i += 2)
                             pk[i >> 1] =
-                                f32_to_bf16_bits(__fmul_rn(__uint_as_float(r[i]), alpha)) |
-                                (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r[i + 1]), alpha)) << 16);
+                                f32_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c][i]), alpha)) |
+                                (f32_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c][i + 1]), alpha)) << 16);
                         uint4 *dst = reinterpret_cast<uint4 *>(cp);
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
@@ -409,16 +419,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         float4 *dst = reinterpret_cast<float4 *>(cp);
 #pragma unroll
                         for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha),
-                                                 __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
-                                                 __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha),
-                                                 __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+                            dst[v] = make_float4(__fmul_rn(__uint_as_float(acc[c][4 * v]), alpha),
+                                                 __fmul_rn(__uint_as_float(acc[c][4 * v + 1]), alpha),
+                                                 __fmul_rn(__uint_as_float(acc[c][4 * v + 2]), alpha),
+                                                 __fmul_rn(__uint_as_float(acc[c][4 * v + 3]), alpha));
                     }
-                }
-                if (have_acc) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(acc_empty);
                 }
             }
             if (have_acc) acc_phase ^= 1u;

@@ -14,13 +14,6 @@ namespace nvfp4moe {
 
 __device__ int32_t g_device_error = 0;
 
-// Byte offset of scale (row r, scale column c) in the MMA layout of a matrix
-// whose rows carry `nsc` scales (nsc % 4 == 0).
-NV_DEV size_t mma_sf_offset(int64_t r, int64_t c, int64_t nsc) {
-    int64_t chunk = (r >> 7) * (nsc >> 2) + (c >> 2);
-    return (size_t)chunk * 512 + (size_t)((r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3));
-}
-
 // ---------------------------------------------------------------------------
 // amax of a bf16 tensor. *amax must be zero before the launch.
 // ---------------------------------------------------------------------------
@@ -54,35 +47,7 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const uint16_t *__restri
 // NVFP4: per-tensor S_enc from amax; one thread quantizes 64 consecutive
 // elements (4 blocks of 16): 128 bytes in, 32 bytes of codes and 4 scales out.
 // ---------------------------------------------------------------------------
-NV_DEV float nvfp4_senc(float amax) {
-    return (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(2688.0f, amax) : 1.0f;
-}
-NV_DEV float nvfp4_ts(float amax) {
-    return (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
-}
-
-// Quantize 16 fp32 values: returns the scale code, writes 8 code bytes (2 words).
-NV_DEV uint32_t nvfp4_block16(const float (&v)[16], float S_enc, uint32_t &w0, uint32_t &w1) {
-    float amax_b = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
-    float t = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S_enc);
-    uint32_t sc = e4m3_encode_pos(t);
-    float sf = e4m3_decode_pos(sc);
-    float enc = (sf == 0.0f) ? 0.0f : __fdiv_rn(S_enc, sf);
-    w0 = 0;
-    w1 = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w0 |= e2m1_encode(__fmul_rn(v[i], enc)) << (4 * i);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w1 |= e2m1_encode(__fmul_rn(v[8 + i], enc)) << (4 * i);
-    return sc;
-}
-
-NV_DEV void unpack8(uint4 q, float *f) {
-    f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x); f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
-    f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z); f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
-}
+NV_DEV void unpack8(uint4 q, float *f) { unpack_bf16x8(q, f); }
 
 // 64 bf16 elements at p -> 32 code bytes at out_codes, 4 scale codes packed in a word.
 NV_DEV uint32_t nvfp4_quant64(const uint16_t *__restrict__ p, float S_enc, uint4 &c0, uint4 &c1) {
@@ -180,8 +145,8 @@ NV_DEV uint32_t mx_block32(const float (&v)[32], uint64_t seed, uint64_t offset,
             for (int j = 0; j < 4; ++j)
                 word |= e4m3_encode_sr(scale_pow2(v[4 * q + j], k), rs[j]) << (8 * j);
         } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) word |= e4m3_encode(scale_pow2(v[4 * q + j], k)) << (8 * j);
+            word = e4m3x2_hw(scale_pow2(v[4 * q], k), scale_pow2(v[4 * q + 1], k)) |
+                   (e4m3x2_hw(scale_pow2(v[4 * q + 2], k), scale_pow2(v[4 * q + 3], k)) << 16);
         }
         w[q] = word;
     }
@@ -214,69 +179,96 @@ __global__ void __launch_bounds__(256) mxfp8_rows_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// MXFP8 along columns, transposed output. A CTA stages a 128-row x 64-column
-// tile in shared memory with coalesced 16-byte loads; thread t quantizes the
-// 32-row block (t / 64) of column (t % 64) and writes its 32 codes as a row
-// of the transposed output.
+// MXFP8 along columns, transposed output. A CTA stages a 128-row x 256-column
+// tile in shared memory with coalesced 16-byte loads. Thread t owns the four
+// adjacent columns 4 * (t % 64) .. +3 of the 32-row block t / 64: those four
+// elements of a row are consecutive in the source, so one Philox call per row
+// gives all four of them their random words.
 // ---------------------------------------------------------------------------
+constexpr int MXC_TR = 128, MXC_TC = 256, MXC_LD = MXC_TC + 8;
+constexpr size_t MXC_SMEM = sizeof(uint16_t) * MXC_TR * MXC_LD;
+
 template <bool SR>
 __global__ void __launch_bounds__(256) mxfp8_cols_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
     uint64_t offset, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int layout) {
-    __shared__ __align__(16) uint16_t tile[128][64 + 8];
-    const int64_t row_tiles = (rows + 127) / 128;
-    const int64_t col_tiles = cols / 64;
+    extern __shared__ __align__(16) uint16_t tile[];
+    const int64_t row_tiles = (rows + MXC_TR - 1) / MXC_TR;
+    const int64_t col_tiles = (cols + MXC_TC - 1) / MXC_TC;
+    const int64_t G = rows / 32;  // scales per output row
     for (int64_t t = blockIdx.x; t < row_tiles * col_tiles; t += gridDim.x) {
-        const int64_t r0 = (t / col_tiles) * 128, c0 = (t % col_tiles) * 64;
-        const int nr = (int)(rows - r0 < 128 ? rows - r0 : 128);
+        const int64_t r0 = (t / col_tiles) * MXC_TR, c0 = (t % col_tiles) * MXC_TC;
+        const int nr = (int)(rows - r0 < MXC_TR ? rows - r0 : MXC_TR);
+        const int nc = (int)(cols - c0 < MXC_TC ? cols - c0 : MXC_TC);
         __syncthreads();
-        for (int v = threadIdx.x; v < 128 * 8; v += 256) {
-            int rr = v >> 3, cc = (v & 7) * 8;
-            uint4 q = rr < nr ? __ldg(reinterpret_cast<const uint4 *>(x + (r0 + rr) * ld + c0 + cc))
-                              : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(&tile[rr][cc]) = q;
+        for (int v = threadIdx.x; v < MXC_TR * (MXC_TC / 8); v += 256) {
+            const int rr = v / (MXC_TC / 8), cc = (v % (MXC_TC / 8)) * 8;
+            uint4 q = make_uint4(0, 0, 0, 0);
+            if (rr < nr && cc < nc) q = __ldg(reinterpret_cast<const uint4 *>(x + (r0 + rr) * ld + c0 + cc));
+            *reinterpret_cast<uint4 *>(&tile[rr * MXC_LD + cc]) = q;
         }
         __syncthreads();
-        const int col = threadIdx.x & 63, rb = threadIdx.x >> 6;
-        if (rb * 32 < nr) {
-            float v[32];
+        const int cl = (threadIdx.x & 63) * 4, rb = threadIdx.x >> 6;
+        if (rb * 32 >= nr || cl >= nc) continue;
+        const uint16_t *tp = tile + (rb * 32) * MXC_LD + cl;
+        float am0 = 0.0f, am1 = 0.0f, am2 = 0.0f, am3 = 0.0f;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const uint2 q = *reinterpret_cast<const uint2 *>(tp + i * MXC_LD);
+            am0 = fmaxf(am0, fabsf(bf16_lo(q.x)));
+            am1 = fmaxf(am1, fabsf(bf16_hi(q.x)));
+            am2 = fmaxf(am2, fabsf(bf16_lo(q.y)));
+            am3 = fmaxf(am3, fabsf(bf16_hi(q.y)));
+        }
+        const int k0 = mx_scale_exp(am0), k1 = mx_scale_exp(am1), k2 = mx_scale_exp(am2),
+                  k3 = mx_scale_exp(am3);
+        const int64_t rbase = r0 + rb * 32, c = c0 + cl;
+        uint32_t w0[8], w1[8], w2[8], w3[8];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float((uint32_t)tile[rb * 32 + i][col] << 16);
-            float amax_b = 0.0f;
+        for (int q = 0; q < 8; ++q) {
+            uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
-            int k = mx_scale_exp(amax_b);
-            const int64_t c = c0 + col, rbase = r0 + rb * 32;
-            uint32_t w[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int i = 4 * q + j;
-                    uint32_t code;
-                    if (SR) {
-                        uint64_t idx = (uint64_t)((rbase + i) * cols + c);
-                        u32x4 r4 = philox_block(seed, offset, idx >> 2);
-                        uint32_t sel = (uint32_t)(idx & 3);
-                        uint32_t rw = sel == 0 ? r4.x : sel == 1 ? r4.y : sel == 2 ? r4.z : r4.w;
-                        code = e4m3_encode_sr(scale_pow2(v[i], k), rw);
-                    } else {
-                        code = e4m3_encode(scale_pow2(v[i], k));
-                    }
-                    word |= code << (8 * j);
+            for (int j = 0; j < 4; ++j) {
+                const int i = 4 * q + j;
+                const uint2 pr = *reinterpret_cast<const uint2 *>(tp + i * MXC_LD);
+                const float v0 = scale_pow2(bf16_lo(pr.x), k0), v1 = scale_pow2(bf16_hi(pr.x), k1);
+                const float v2 = scale_pow2(bf16_lo(pr.y), k2), v3 = scale_pow2(bf16_hi(pr.y), k3);
+                uint32_t e0, e1, e2, e3;
+                if (SR) {
+                    // elements (rbase + i, c .. c + 3): row-major index multiple of 4
+                    const u32x4 r4 = philox_block(seed, offset, (uint64_t)((rbase + i) * cols + c) >> 2);
+                    e0 = e4m3_encode_sr(v0, r4.x);
+                    e1 = e4m3_encode_sr(v1, r4.y);
+                    e2 = e4m3_encode_sr(v2, r4.z);
+                    e3 = e4m3_encode_sr(v3, r4.w);
+                } else {
+                    const uint32_t p01 = e4m3x2_hw(v0, v1), p23 = e4m3x2_hw(v2, v3);
+                    e0 = p01 & 0xFFu; e1 = p01 >> 8; e2 = p23 & 0xFFu; e3 = p23 >> 8;
                 }
-                w[q] = word;
+                a0 |= e0 << (8 * j);
+                a1 |= e1 << (8 * j);
+                a2 |= e2 << (8 * j);
+                a3 |= e3 << (8 * j);
             }
-            uint4 *co = reinterpret_cast<uint4 *>(codes + c * rows + rbase);
-            co[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            co[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            const int64_t G = rows / 32;
-            const int64_t b = rbase / 32;
+            w0[q] = a0; w1[q] = a1; w2[q] = a2; w3[q] = a3;
+        }
+        uint4 *o0 = reinterpret_cast<uint4 *>(codes + (c + 0) * rows + rbase);
+        uint4 *o1 = reinterpret_cast<uint4 *>(codes + (c + 1) * rows + rbase);
+        uint4 *o2 = reinterpret_cast<uint4 *>(codes + (c + 2) * rows + rbase);
+        uint4 *o3 = reinterpret_cast<uint4 *>(codes + (c + 3) * rows + rbase);
+        o0[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]); o0[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
+        o1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]); o1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+        o2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]); o2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+        o3[0] = make_uint4(w3[0], w3[1], w3[2], w3[3]); o3[1] = make_uint4(w3[4], w3[5], w3[6], w3[7]);
+        const int64_t b = rbase / 32;
+        const int ks[4] = {k0, k1, k2, k3};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint8_t e8 = (uint8_t)(ks[j] + 127);
             if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
-                scales[c * G + b] = (uint8_t)(k + 127);
+                scales[(c + j) * G + b] = e8;
             else
-                scales[mma_sf_offset(c, b, G)] = (uint8_t)(k + 127);
+                scales[mma_sf_offset(c + j, b, G)] = e8;
         }
     }
 }
@@ -378,12 +370,9 @@ __global__ void __launch_bounds__(256) rht32_quant_kernel(
         float v[32];
         rht32_fwd(x + r * ld + b * 32, signs, v);
         if (fmt == NVFP4MOE_FMT_NVFP4) {
-            float h0[16], h1[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) { h0[j] = v[j]; h1[j] = v[16 + j]; }
             uint32_t w0, w1, w2, w3;
-            uint32_t s0 = nvfp4_block16(h0, S_enc, w0, w1);
-            uint32_t s1 = nvfp4_block16(h1, S_enc, w2, w3);
+            uint32_t s0 = nvfp4_block16(v, S_enc, w0, w1);
+            uint32_t s1 = nvfp4_block16(v + 16, S_enc, w2, w3);
             *reinterpret_cast<uint4 *>(codes + r * (cols / 2) + b * 16) = make_uint4(w0, w1, w2, w3);
             *reinterpret_cast<uint16_t *>(scales + r * (cols / 16) + b * 2) =
                 (uint16_t)(s0 | (s1 << 8));
@@ -502,14 +491,25 @@ cudaError_t launch_mxfp8_quantize(const uint16_t *x, int64_t rows, int64_t cols,
             mxfp8_rows_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes,
                                                        scales, layout);
     } else {
-        int64_t tiles = ((rows + 127) / 128) * (cols / 64);
-        int g = (int)(tiles < 148 * 8 ? tiles : 148 * 8);
+        static bool attr = false;
+        if (!attr) {
+            cudaError_t e = cudaFuncSetAttribute(mxfp8_cols_kernel<true>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)MXC_SMEM);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(mxfp8_cols_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MXC_SMEM);
+            if (e != cudaSuccess) return e;
+            attr = true;
+        }
+        int64_t tiles = ((rows + MXC_TR - 1) / MXC_TR) * ((cols + MXC_TC - 1) / MXC_TC);
+        int g = (int)(tiles < 148 * 3 ? tiles : 148 * 3);
         if (sr)
-            mxfp8_cols_kernel<true><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes, scales,
-                                                      layout);
+            mxfp8_cols_kernel<true><<<g, 256, MXC_SMEM, s>>>(x, rows, cols, ld, seed, offset, codes,
+                                                             scales, layout);
         else
-            mxfp8_cols_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes,
-                                                       scales, layout);
+            mxfp8_cols_kernel<false><<<g, 256, MXC_SMEM, s>>>(x, rows, cols, ld, seed, offset,
+                                                              codes, scales, layout);
     }
     return cudaGetLastError();
 }
@@ -590,6 +590,47 @@ cudaError_t launch_nvfp4_quant_grouped(const uint16_t *x, int64_t rows_alloc, in
     int g = grid_for(rows_alloc * (cols / 64));
     nvfp4_quant_grouped_kernel<<<g, 256, (E + 1) * sizeof(int32_t), s>>>(x, cols, off, E, amax,
                                                                          codes, scales, ts);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Self-test of the hardware conversions the quantizers use: every finite fp32
+// input, hardware result against the library's software encoders.
+// which 0: cvt.rn.satfinite.e2m1x2.f32; which 1: cvt.rn.satfinite.e4m3x2.f32.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) selftest_cvt_kernel(int which,
+                                                           unsigned long long *mismatches) {
+    unsigned long long bad = 0;
+    const uint64_t groups = 1ull << 29;  // 8 consecutive bit patterns per group
+    for (uint64_t g = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; g < groups;
+         g += (uint64_t)gridDim.x * blockDim.x) {
+        const uint32_t base = (uint32_t)(g << 3);
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(base + j);
+        if (which == 0) {
+            const uint32_t hw = e2m1x8_hw(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (isfinite(v[j]) && ((hw >> (4 * j)) & 15u) != e2m1_encode(v[j])) ++bad;
+        } else {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const uint32_t hw = e4m3x2_hw(v[2 * p], v[2 * p + 1]);
+                if (isfinite(v[2 * p]) && (hw & 0xFFu) != e4m3_encode(v[2 * p])) ++bad;
+                if (isfinite(v[2 * p + 1]) && (hw >> 8) != e4m3_encode(v[2 * p + 1])) ++bad;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xFFFFFFFFu, bad, o);
+    if ((threadIdx.x & 31) == 0 && bad) atomicAdd(mismatches, bad);
+}
+
+cudaError_t launch_selftest(int which, unsigned long long *mismatches, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), s);
+    if (e != cudaSuccess) return e;
+    selftest_cvt_kernel<<<148 * 8, 256, 0, s>>>(which, mismatches);
     return cudaGetLastError();
 }
 

@@ -32,6 +32,8 @@ cudaError_t launch_nvfp4_quant_grouped(const uint16_t *x, int64_t rows_alloc, in
                                        uint8_t *codes, uint8_t *scales, float *ts,
                                        cudaStream_t s);
 
+cudaError_t launch_selftest(int which, unsigned long long *mismatches, cudaStream_t s);
+
 // routing / permutation / combine (route.cu)
 size_t route_permute_ws_bytes(int64_t T, int32_t E, int32_t k);
 cudaError_t launch_route_permute(const float *logits, const uint16_t *x, int64_t T, int32_t E,

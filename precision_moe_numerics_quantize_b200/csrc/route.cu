@@ -19,11 +19,6 @@ namespace nvfp4moe {
 
 static constexpr int CHUNK = 1024;
 
-NV_DEV size_t mma_sf_off(int64_t r, int64_t c, int64_t nsc) {
-    int64_t chunk = (r >> 7) * (nsc >> 2) + (c >> 2);
-    return (size_t)chunk * 512 + (size_t)((r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3));
-}
-
 // ---------------------------------------------------------------------------
 // 1. top-k: each lane owns experts lane, lane + 32, ...; k rounds of a warp
 // argmax (largest logit, ties to the lower expert id).
@@ -206,41 +201,14 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t *__restrict_
 // 5. quantize token rows once and copy to their k destination rows; zero the
 // padding rows of every expert.
 // ---------------------------------------------------------------------------
-NV_DEV float senc_of(float amax) {
-    return (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(2688.0f, amax) : 1.0f;
-}
-
-NV_DEV void unpack8r(uint4 q, float *f) {
-    f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x); f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
-    f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z); f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
-}
-
-NV_DEV uint32_t quant_block16(const float (&v)[16], float S_enc, uint32_t &w0, uint32_t &w1) {
-    float amax_b = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
-    float t = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S_enc);
-    uint32_t sc = e4m3_encode_pos(t);
-    float sf = e4m3_decode_pos(sc);
-    float enc = (sf == 0.0f) ? 0.0f : __fdiv_rn(S_enc, sf);
-    w0 = 0;
-    w1 = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w0 |= e2m1_encode(__fmul_rn(v[i], enc)) << (4 * i);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w1 |= e2m1_encode(__fmul_rn(v[8 + i], enc)) << (4 * i);
-    return sc;
-}
-
 __global__ void __launch_bounds__(256) dispatch_quant_kernel(
     const uint16_t *__restrict__ x, int64_t T, int64_t d, int32_t k,
     const float *__restrict__ amax_p, const int32_t *__restrict__ pos,
     uint8_t *__restrict__ xq, uint8_t *__restrict__ xq_sc, float *__restrict__ x_ts,
     int write_ts) {
     const float amax = *amax_p;
-    const float S_enc = senc_of(amax);
-    if (write_ts && blockIdx.x == 0 && threadIdx.x == 0)
-        *x_ts = (amax > 0.0f && amax <= 3.402823466e38f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    const float S_enc = nvfp4_senc(amax);
+    if (write_ts && blockIdx.x == 0 && threadIdx.x == 0) *x_ts = nvfp4_ts(amax);
     const int64_t G = d / 64;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < T * G;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -250,9 +218,9 @@ __global__ void __launch_bounds__(256) dispatch_quant_kernel(
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
             float v[16];
-            unpack8r(__ldg(pv + 2 * b), v);
-            unpack8r(__ldg(pv + 2 * b + 1), v + 8);
-            scw |= quant_block16(v, S_enc, w[2 * b], w[2 * b + 1]) << (8 * b);
+            unpack_bf16x8(__ldg(pv + 2 * b), v);
+            unpack_bf16x8(__ldg(pv + 2 * b + 1), v + 8);
+            scw |= nvfp4_block16(v, S_enc, w[2 * b], w[2 * b + 1]) << (8 * b);
         }
         const uint4 c0 = make_uint4(w[0], w[1], w[2], w[3]);
         const uint4 c1 = make_uint4(w[4], w[5], w[6], w[7]);
@@ -261,7 +229,7 @@ __global__ void __launch_bounds__(256) dispatch_quant_kernel(
             uint4 *co = reinterpret_cast<uint4 *>(xq + row * (d / 2) + g * 32);
             co[0] = c0;
             co[1] = c1;
-            *reinterpret_cast<uint32_t *>(xq_sc + mma_sf_off(row, g * 4, d / 16)) = scw;
+            *reinterpret_cast<uint32_t *>(xq_sc + mma_sf_offset(row, g * 4, d / 16)) = scw;
         }
     }
 }
@@ -278,7 +246,7 @@ __global__ void __launch_bounds__(256) zero_pad_rows_kernel(
         uint4 *co = reinterpret_cast<uint4 *>(xq + r * (d / 2) + g * 32);
         co[0] = make_uint4(0, 0, 0, 0);
         co[1] = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint32_t *>(xq_sc + mma_sf_off(r, g * 4, d / 16)) = 0u;
+        *reinterpret_cast<uint32_t *>(xq_sc + mma_sf_offset(r, g * 4, d / 16)) = 0u;
     }
 }
 

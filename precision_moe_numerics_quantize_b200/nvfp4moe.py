@@ -42,6 +42,7 @@ _SIGS = {
     "nvfp4moe_last_error": (C.c_char_p, []),
     "nvfp4moe_device_error": (C.c_int, [_P]),
     "nvfp4moe_max_rows": (_I64, [_I64, _I32, _I32]),
+    "nvfp4moe_selftest": (C.c_int, [_I, _P, _P]),
     "nvfp4moe_amax_bf16": (C.c_int, [_P, _I64, _I64, _I64, _P, _P]),
     "nvfp4_quantize": (C.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P]),
     "nvfp4_dequantize": (C.c_int, [_P, _P, _P, _I64, _I64, _I, _P, _P]),
@@ -112,6 +113,11 @@ def device_error():
     code = C.c_int32(0)
     st = lib().nvfp4moe_device_error(C.byref(code))
     return st, code.value
+
+
+def selftest(which, mismatches, stream=None):
+    """Exhaustive hardware-conversion check; mismatch count in mismatches (int64 [1])."""
+    _check("nvfp4moe_selftest", lib().nvfp4moe_selftest(which, _ptr(mismatches), _stream(stream)))
 
 
 def max_rows(T, k, E):

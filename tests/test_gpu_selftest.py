@@ -1,0 +1,16 @@
+"""The hardware conversions used by the quantizers (cvt.rn.satfinite to E2M1
+pairs and to E4M3 pairs) agree with the library's software encoders on every
+finite fp32 input. The software encoders are the ones the parity tests pin to
+the oracle, so this extends that pin to the hardware path over all inputs."""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_hardware_conversion_matches_encoder_on_all_fp32(dev, lib, which):
+    bad = torch.full((1,), -1, dtype=torch.int64, device=dev)
+    lib.selftest(which, bad)
+    torch.cuda.synchronize()
+    assert bad.item() == 0
