@@ -5,23 +5,32 @@
 // minor, so neighbouring CTAs share the weight tile through L2. The tile list
 // is derived on the device from the group offsets: no host synchronisation.
 //
-// Roles (320 threads):
-//   warp 0      TMA producer: per 128-byte K stage, the A tile (128 rows),
-//               the B tile (two 128-row halves) with 128-byte swizzle, and
-//               the block scales (already stored in the MMA layout) with
-//               plain bulk copies. STAGES-deep mbarrier ring.
-//   warp 1      MMA issuer (one thread): copies the stage's scales from shared
-//               memory to TMEM (tcgen05.cp 32x128b.warpx4), then issues four
-//               block-scaled MMAs (kind::mxf4nvf4 block16 for NVFP4 operands,
-//               kind::mxf8f6f4 with E8M0 scales for MXFP8), accumulating in
-//               TMEM; tcgen05.commit frees the stage and finally signals the
-//               accumulator.
-//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (warp w reads
-//               lanes 32*(w%4)..+31; two warps per lane quarter split the
-//               columns), scaling by the per-group alpha, then either SwiGLU
-//               with a fused per-group amax (gate/up halves of the B tile)
-//               or a plain bf16 / fp32 store.
-// TMEM: columns [0, 256) accumulator, [256, 288) A scales, [288, 320) B scales.
+// Roles (448 threads, 14 warps):
+//   warp 0       TMA producer: per 128-byte K stage, the A tile (128 rows),
+//                the B tile (two 128-row halves) with 128-byte swizzle, and
+//                the block scales (stored in the MMA chunk layout) with plain
+//                bulk copies. STAGES-deep mbarrier ring.
+//   warps 2..5   scale warps, one per TMEM lane quarter: they move each stage's
+//                scales from shared memory into a TMEM ring with tcgen05.st,
+//                in the replicated layout the block-scaled MMA reads (lane r of
+//                every quarter holds the scales of rows r, r+32, r+64, ...).
+//                Doing this with thread stores rather than tcgen05.cp keeps the
+//                tensor pipe for MMAs only: a tcgen05.cp occupies the in-order
+//                tensor pipe about as long as an MMA.
+//   warp 1       MMA issuer (one thread): four block-scaled MMAs per stage
+//                (kind::mxf4nvf4 block16 for NVFP4, kind::mxf8f6f4 with E8M0
+//                scales for MXFP8) into the TMEM accumulator; tcgen05.commit
+//                frees the stage and finally signals the accumulator.
+//   warps 6..13  epilogue: tcgen05.ld of the fp32 accumulator (warp w reads
+//                lanes 32*(w%4)..+31, two warps per quarter split the columns),
+//                released back to the MMA warp as soon as it is in registers;
+//                then SwiGLU with a fused per-group amax, or a bf16 / fp32 store.
+// TMEM: columns [0, 256) accumulator, [256, 512) scale ring, 64 columns per
+// stage: B scales of MMA kb at +8kb .. +8kb+7 (every lane quarter holds all 256
+// B rows); A scales of MMA kb at the 4-column group +32+4kb (lane quarter q,
+// which computes rows 32q..32q+31, reads column +32+4kb+q, so each quarter
+// writes only that one column). Scale addresses given to the MMA and the
+// column of every multi-column tcgen05.st stay 4-column aligned.
 //
 // Every wait is bounded (about 2 s); a wait that runs out records its id in
 // the device error word, raises a CTA-wide abort flag and the kernel winds
@@ -39,16 +48,18 @@ constexpr int BM = 128, BN = 256, KBYTES = 128, STAGES = 4;
 constexpr int A_STAGE = BM * KBYTES;   // 16 KB
 constexpr int B_STAGE = BN * KBYTES;   // 32 KB
 constexpr int SFA_STAGE = 2048, SFB_STAGE = 4096;
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 448;
 constexpr int MAX_GROUPS = 1024;
-constexpr uint32_t TMEM_COLS = 512, TMEM_SFA = 256, TMEM_SFB = 288;
+constexpr uint32_t TMEM_COLS = 512, TMEM_SF = 256, SF_SLOT_COLS = 64;
 
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;      // full[S], empty[S], acc_full, acc_empty
-constexpr int OFF_MISC = OFF_BAR + 8 * (2 * STAGES + 2);   // tmem base, abort flag, total tiles
+// barriers: full[S] (operands), sf_loaded[S] (scales in smem), sf_full[S]
+// (scales in TMEM), empty[S], acc_full, acc_empty
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int OFF_MISC = OFF_BAR + 8 * (4 * STAGES + 2);  // tmem base, abort flag
 constexpr int OFF_PREFIX = OFF_MISC + 16;
 constexpr int SMEM_BYTES = OFF_PREFIX + 4 * (MAX_GROUPS + 1);
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
@@ -166,7 +177,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *empty = full + STAGES;
-    uint64_t *acc_full = empty + STAGES;
+    uint64_t *sf_full = empty + STAGES;
+    uint64_t *sf_loaded = sf_full + STAGES;
+    uint64_t *acc_full = sf_loaded + STAGES;
     uint64_t *acc_empty = acc_full + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int32_t *abort_flag = reinterpret_cast<int32_t *>(smem + OFF_MISC + 4);
@@ -193,7 +206,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     __syncthreads();
     if (warp == 0) {
-        // inclusive scan of prefix[1..G] in chunks of 32 per lane
+        // inclusive scan of prefix[1..G] in chunks of `per` entries per lane
         const int per = (G + 31) / 32;
         int32_t s = 0;
         for (int i = 0; i < per; ++i) {
@@ -222,6 +235,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_full[s], 4);
+            mbar_init(&sf_loaded[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 8);
@@ -234,7 +249,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int64_t total = prefix[G];
     const bool nvf4 = p.kind == 0;
     const uint32_t sfa_bytes = nvf4 ? 2048u : 512u;  // per 128-row block per stage
-    const uint32_t stage_tx = A_STAGE + B_STAGE + 3 * sfa_bytes;
+    const uint32_t op_tx = A_STAGE + B_STAGE;
 
     if (warp == 0) {
         // ======================= TMA producer =======================
@@ -247,25 +262,76 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const Tile T = tile_info(p, prefix, t);
                 for (int kt = 0; kt < T.kt; ++kt) {
                     if (!wait_or_abort(&empty[s], phase ^ 1u, abort_flag, WAIT_GEMM_EMPTY)) break;
-                    mbar_arrive_expect_tx(&full[s], stage_tx);
-                    const int32_t kx = (int32_t)(T.k0 + (int64_t)kt * 128);  // byte column
-                    uint8_t *sa = smem + OFF_A + s * A_STAGE;
-                    uint8_t *sb = smem + OFF_B + s * B_STAGE;
-                    tma_load_2d(sa, &tmA, kx, (int32_t)T.a_row, &full[s]);
-                    tma_load_2d(sb, &tmB, kx, (int32_t)T.b_row0, &full[s]);
-                    tma_load_2d(sb + B_STAGE / 2, &tmB, kx, (int32_t)T.b_row1, &full[s]);
-                    // scales: NVFP4 stage = 4 chunks (256 K) per 128 rows; MXFP8 = 1 chunk (128 K)
+                    // scales first, on their own barrier: they are small, land
+                    // early, and the scale warps move them into TMEM while the
+                    // operand tiles are still in flight
+                    // (NVFP4 stage = 4 chunks (256 K) per 128 rows; MXFP8 = 1 chunk (128 K))
                     const int64_t kc = nvf4 ? (int64_t)kt * 4 : (T.k0 / 128 + kt);
                     const uint8_t *srcA = p.a_sc + ((T.a_row / 128) * p.a_nkc + kc) * 512;
                     const uint8_t *srcB0 = p.b_sc + ((T.b_row0 / 128) * p.b_nkc + kc) * 512;
                     const uint8_t *srcB1 = p.b_sc + ((T.b_row1 / 128) * p.b_nkc + kc) * 512;
                     uint8_t *ssfa = smem + OFF_SFA + s * SFA_STAGE;
                     uint8_t *ssfb = smem + OFF_SFB + s * SFB_STAGE;
-                    bulk_load(ssfa, srcA, sfa_bytes, &full[s]);
-                    bulk_load(ssfb, srcB0, sfa_bytes, &full[s]);
-                    bulk_load(ssfb + sfa_bytes, srcB1, sfa_bytes, &full[s]);
+                    mbar_arrive_expect_tx(&sf_loaded[s], 3 * sfa_bytes);
+                    bulk_load(ssfa, srcA, sfa_bytes, &sf_loaded[s]);
+                    bulk_load(ssfb, srcB0, sfa_bytes, &sf_loaded[s]);
+                    bulk_load(ssfb + sfa_bytes, srcB1, sfa_bytes, &sf_loaded[s]);
+                    mbar_arrive_expect_tx(&full[s], op_tx);
+                    const int32_t kx = (int32_t)(T.k0 + (int64_t)kt * 128);  // byte column
+                    uint8_t *sa = smem + OFF_A + s * A_STAGE;
+                    uint8_t *sb = smem + OFF_B + s * B_STAGE;
+                    tma_load_2d(sa, &tmA, kx, (int32_t)T.a_row, &full[s]);
+                    tma_load_2d(sb, &tmB, kx, (int32_t)T.b_row0, &full[s]);
+                    tma_load_2d(sb + B_STAGE / 2, &tmB, kx, (int32_t)T.b_row1, &full[s]);
                     if (++s == STAGES) { s = 0; phase ^= 1u; }
                 }
+            }
+        }
+    } else if (warp >= 2 && warp <= 5) {
+        // ======================= scale warps =======================
+        // In a 512-byte scale chunk the word (4 scales) of row r0 + 32 r1 sits
+        // at byte r0 * 16 + r1 * 4, so lane r0 reads 16 contiguous bytes per
+        // chunk: the B words of tile rows r0 + 32 j, and from the A chunk the
+        // word of row r0 + 32 q, the only A row this lane quarter computes.
+        const int q = warp & 3;
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+        int s = 0;
+        uint32_t phase = 0;
+        for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+            const Tile T = tile_info(p, prefix, t);
+            for (int kt = 0; kt < T.kt; ++kt) {
+                if (!wait_or_abort(&sf_loaded[s], phase, abort_flag, WAIT_GEMM_FULL)) break;
+                const uint8_t *ssfa = smem + OFF_SFA + s * SFA_STAGE;
+                const uint8_t *ssfb = smem + OFF_SFB + s * SFB_STAGE;
+                const uint32_t slot = lane_addr + TMEM_SF + s * SF_SLOT_COLS;
+                if (nvf4) {
+                    uint32_t b[32], a[4];
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        const uint4 b0 = *reinterpret_cast<const uint4 *>(ssfb + kb * 512 + lane * 16);
+                        const uint4 b1 = *reinterpret_cast<const uint4 *>(ssfb + 2048 + kb * 512 + lane * 16);
+                        b[8 * kb + 0] = b0.x; b[8 * kb + 1] = b0.y; b[8 * kb + 2] = b0.z; b[8 * kb + 3] = b0.w;
+                        b[8 * kb + 4] = b1.x; b[8 * kb + 5] = b1.y; b[8 * kb + 6] = b1.z; b[8 * kb + 7] = b1.w;
+                        a[kb] = *reinterpret_cast<const uint32_t *>(ssfa + kb * 512 + lane * 16 + q * 4);
+                    }
+                    tmem_st_32x32b_x32(slot, b);
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) tmem_st_32x32b_x1(slot + 32 + 4 * kb + q, a[kb]);
+                } else {
+                    // one chunk per stage: the four scale bytes of a word serve
+                    // the four MMAs (byte kb selected by the MMA's scale id)
+                    const uint4 b0 = *reinterpret_cast<const uint4 *>(ssfb + lane * 16);
+                    const uint4 b1 = *reinterpret_cast<const uint4 *>(ssfb + 512 + lane * 16);
+                    const uint32_t b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    tmem_st_32x32b_x8(slot, b);
+                    tmem_st_32x32b_x1(slot + 32 + q,
+                                      *reinterpret_cast<const uint32_t *>(ssfa + lane * 16 + q * 4));
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_full[s]);
+                if (++s == STAGES) { s = 0; phase ^= 1u; }
             }
         }
     } else if (warp == 1) {
@@ -281,42 +347,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < T.kt; ++kt) {
-                    if (!wait_or_abort(&full[s], phase, abort_flag, WAIT_GEMM_FULL)) { ok = false; break; }
+                    if (!wait_or_abort(&full[s], phase, abort_flag, WAIT_GEMM_FULL) ||
+                        !wait_or_abort(&sf_full[s], phase, abort_flag, WAIT_GEMM_FULL)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + OFF_A + s * A_STAGE);
                     const uint32_t sb = smem_u32(smem + OFF_B + s * B_STAGE);
-                    const uint32_t ssfa = smem_u32(smem + OFF_SFA + s * SFA_STAGE);
-                    const uint32_t ssfb = smem_u32(smem + OFF_SFB + s * SFB_STAGE);
-                    if (nvf4) {
+                    const uint32_t sf = tmem_base + TMEM_SF + s * SF_SLOT_COLS;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            tc_cp_32x128b_warpx4(tmem_base + TMEM_SFA + 4 * c,
-                                                 smem_desc(ssfa + 512 * c, 0, 128, 0));
-                            tc_cp_32x128b_warpx4(tmem_base + TMEM_SFB + 8 * c,
-                                                 smem_desc(ssfb + 512 * c, 0, 128, 0));
-                            tc_cp_32x128b_warpx4(tmem_base + TMEM_SFB + 8 * c + 4,
-                                                 smem_desc(ssfb + 2048 + 512 * c, 0, 128, 0));
-                        }
-#pragma unroll
-                        for (int kb = 0; kb < 4; ++kb) {
-                            const uint64_t ad = smem_desc(sa + 32 * kb, 16, 1024, 2);
-                            const uint64_t bd = smem_desc(sb + 32 * kb, 16, 1024, 2);
-                            tc_mma_nvf4(d_tmem, ad, bd, idesc_nvf4(), tmem_base + TMEM_SFA + 4 * kb,
-                                        tmem_base + TMEM_SFB + 8 * kb, (kt | kb) != 0);
-                        }
-                    } else {
-                        tc_cp_32x128b_warpx4(tmem_base + TMEM_SFA, smem_desc(ssfa, 0, 128, 0));
-                        tc_cp_32x128b_warpx4(tmem_base + TMEM_SFB, smem_desc(ssfb, 0, 128, 0));
-                        tc_cp_32x128b_warpx4(tmem_base + TMEM_SFB + 4,
-                                             smem_desc(ssfb + 512, 0, 128, 0));
-#pragma unroll
-                        for (int kb = 0; kb < 4; ++kb) {
-                            const uint64_t ad = smem_desc(sa + 32 * kb, 16, 1024, 2);
-                            const uint64_t bd = smem_desc(sb + 32 * kb, 16, 1024, 2);
-                            const uint32_t sub = (uint32_t)kb << 30;  // byte kb of the scale word
-                            tc_mma_mxf8(d_tmem, ad, bd, idesc_mxf8((uint32_t)kb),
-                                        (tmem_base + TMEM_SFA) | sub, (tmem_base + TMEM_SFB) | sub,
+                    for (int kb = 0; kb < 4; ++kb) {
+                        const uint64_t ad = smem_desc(sa + 32 * kb, 16, 1024, 2);
+                        const uint64_t bd = smem_desc(sb + 32 * kb, 16, 1024, 2);
+                        if (nvf4) {
+                            tc_mma_nvf4(d_tmem, ad, bd, idesc_nvf4(), sf + 32 + 4 * kb, sf + 8 * kb,
                                         (kt | kb) != 0);
+                        } else {
+                            const uint32_t sub = (uint32_t)kb << 30;  // byte kb of the scale word
+                            tc_mma_mxf8(d_tmem, ad, bd, idesc_mxf8((uint32_t)kb), (sf + 32) | sub,
+                                        sf | sub, (kt | kb) != 0);
                         }
                     }
                     tc_commit(&empty[s]);
@@ -330,8 +377,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else {
         // ======================= epilogue =======================
         const int q = warp & 3;          // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;
+        const int half = (warp - 6) >> 2;
         const int row_in_tile = q * 32 + lane;
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
         uint32_t acc_phase = 0;
         for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
             const Tile T = tile_info(p, prefix, t);
@@ -343,86 +391,117 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (!wait_or_abort(acc_full, acc_phase, abort_flag, WAIT_GEMM_ACC_FULL)) break;
                 tc_fence_after();
             }
-            const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
-            // Drain this warp's 128 accumulator columns into registers, hand the
-            // accumulator back to the MMA warp at once, then do the math and the
-            // stores while the next tile's MMAs run.
-            uint32_t acc[4][32];
-            if (have_acc) {
-                if (p.epi == EPI_SWIGLU_AMAX) {
-                    tmem_ld_32x32b_x32(lane_addr + half * 64, acc[0]);           // gate
-                    tmem_ld_32x32b_x32(lane_addr + half * 64 + 32, acc[1]);
-                    tmem_ld_32x32b_x32(lane_addr + 128 + half * 64, acc[2]);     // up
-                    tmem_ld_32x32b_x32(lane_addr + 128 + half * 64 + 32, acc[3]);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        tmem_ld_32x32b_x32(lane_addr + half * 128 + c * 32, acc[c]);
-                }
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c][i] = 0u;
-            }
             if (p.epi == EPI_SWIGLU_AMAX) {
+                // two rounds of (32 gate + 32 up) columns; the accumulator goes
+                // back to the MMA warp once the second round is in registers
                 uint16_t *h = static_cast<uint16_t *>(p.c);
                 float amax = 0.0f;
+                uint32_t pk[2][16];
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int hc = half * 64 + c * 32;
-                    uint32_t pk[16];
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32b_x32(lane_addr + hc, g);
+                    tmem_ld_32x32b_x32(lane_addr + 128 + hc, u);
+                    tmem_wait_ld();
+                    if (c == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acc_empty);
+                    }
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         float hv[2];
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            const float gq = __fmul_rn(__uint_as_float(acc[c][i + j]), alpha);
-                            const float uq = __fmul_rn(__uint_as_float(acc[2 + c][i + j]), alpha);
+                            const float gq = __fmul_rn(__uint_as_float(g[i + j]), alpha);
+                            const float uq = __fmul_rn(__uint_as_float(u[i + j]), alpha);
                             const float den = fminf(1.0f + __expf(-gq), 1e30f);
                             hv[j] = __fmul_rn(__fdividef(gq, den), uq);
                         }
                         const uint32_t b0 = f32_to_bf16_bits(hv[0]), b1 = f32_to_bf16_bits(hv[1]);
                         amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(b0 << 16)),
                                                  fabsf(__uint_as_float(b1 << 16))));
-                        pk[i >> 1] = b0 | (b1 << 16);
+                        pk[c][i >> 1] = b0 | (b1 << 16);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(h + row * p.ldc + T.out_col + hc);
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(h + row * p.ldc + T.out_col + half * 64 + c * 32);
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        dst[v] = make_uint4(pk[c][4 * v], pk[c][4 * v + 1], pk[c][4 * v + 2], pk[c][4 * v + 3]);
                 }
                 amax = warp_max(amax);
                 if (lane == 0) atomic_max_nonneg(p.amax + T.g, amax);
-            } else {
+            } else if (p.epi == EPI_STORE_BF16) {
+                // two rounds of 64 columns, converted to bf16 as they arrive
+                uint32_t pk[4][16];
+#pragma unroll
+                for (int rd = 0; rd < 2; ++rd) {
+                    uint32_t r0[32], r1[32];
+                    if (have_acc) {
+                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64, r0);
+                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64 + 32, r1);
+                        tmem_wait_ld();
+                        if (rd == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(acc_empty);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0u;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        pk[2 * rd][i >> 1] =
+                            f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[i]), alpha)) |
+                            (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[i + 1]), alpha)) << 16);
+                        pk[2 * rd + 1][i >> 1] =
+                            f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[i]), alpha)) |
+                            (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[i + 1]), alpha)) << 16);
+                    }
+                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const int col = half * 128 + c * 32;
-                    if (p.epi == EPI_STORE_BF16) {
-                        uint16_t *cp = static_cast<uint16_t *>(p.c) + row * p.ldc + T.out_col + col;
-                        uint32_t pk[16];
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.c) + row * p.ldc +
+                                                           T.out_col + half * 128 + c * 32);
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2)
-                            pk[i >> 1] =
-                                f32_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c][i]), alpha)) |
-                                (f32_to_bf16_bits(__fmul_rn(__uint_as_float(acc[c][i + 1]), alpha)) << 16);
-                        uint4 *dst = reinterpret_cast<uint4 *>(cp);
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(pk[c][4 * v], pk[c][4 * v + 1], pk[c][4 * v + 2], pk[c][4 * v + 3]);
+                }
+            } else {
+                // fp32 out: two rounds of 64 columns stored as they arrive
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                for (int rd = 0; rd < 2; ++rd) {
+                    uint32_t r0[32], r1[32];
+                    if (have_acc) {
+                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64, r0);
+                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64 + 32, r1);
+                        tmem_wait_ld();
+                        if (rd == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(acc_empty);
+                        }
                     } else {
-                        float *cp = static_cast<float *>(p.c) + row * p.ldc + T.out_col + col;
-                        float4 *dst = reinterpret_cast<float4 *>(cp);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__fmul_rn(__uint_as_float(acc[c][4 * v]), alpha),
-                                                 __fmul_rn(__uint_as_float(acc[c][4 * v + 1]), alpha),
-                                                 __fmul_rn(__uint_as_float(acc[c][4 * v + 2]), alpha),
-                                                 __fmul_rn(__uint_as_float(acc[c][4 * v + 3]), alpha));
+                        for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0u;
+                    }
+                    float *cp = static_cast<float *>(p.c) + row * p.ldc + T.out_col + half * 128 + rd * 64;
+                    float4 *d0 = reinterpret_cast<float4 *>(cp);
+                    float4 *d1 = reinterpret_cast<float4 *>(cp + 32);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        d0[v] = make_float4(__fmul_rn(__uint_as_float(r0[4 * v]), alpha),
+                                            __fmul_rn(__uint_as_float(r0[4 * v + 1]), alpha),
+                                            __fmul_rn(__uint_as_float(r0[4 * v + 2]), alpha),
+                                            __fmul_rn(__uint_as_float(r0[4 * v + 3]), alpha));
+                        d1[v] = make_float4(__fmul_rn(__uint_as_float(r1[4 * v]), alpha),
+                                            __fmul_rn(__uint_as_float(r1[4 * v + 1]), alpha),
+                                            __fmul_rn(__uint_as_float(r1[4 * v + 2]), alpha),
+                                            __fmul_rn(__uint_as_float(r1[4 * v + 3]), alpha));
                     }
                 }
             }
