@@ -169,6 +169,7 @@ nvfp4moe_status nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, in
          "nvfp4_quantize: cols %% 64 == 0, ld %% 8 == 0, ld >= cols required");
     nvfp4moe_status st = check_layout(layout, rows, cols / 16, "nvfp4_quantize");
     if (st) return st;
+    NEED(rows * (cols / 64) < (1LL << 31), NVFP4MOE_ERR_SHAPE, "nvfp4_quantize: tensor too large");
     if (rows * cols) {
         NEED_PTR(x);
         NEED_PTR(codes);
@@ -209,6 +210,7 @@ nvfp4moe_status mxfp8_quantize_sr(const uint16_t *x, int64_t rows, int64_t cols,
     NEED(rounding == NVFP4MOE_ROUND_RNE || rounding == NVFP4MOE_ROUND_SR,
          NVFP4MOE_ERR_INVALID_ARG, "mxfp8_quantize_sr: bad rounding %d", rounding);
     NEED(ld % 8 == 0 && ld >= cols, NVFP4MOE_ERR_SHAPE, "mxfp8_quantize_sr: ld %% 8 == 0, ld >= cols");
+    NEED(rows * (cols / 32 + 1) < (1LL << 31), NVFP4MOE_ERR_SHAPE, "mxfp8_quantize_sr: tensor too large");
     if (axis == 0) {
         NEED(cols % 32 == 0, NVFP4MOE_ERR_SHAPE, "mxfp8_quantize_sr: axis 0 needs cols %% 32 == 0");
         nvfp4moe_status st = check_layout(layout, rows, cols / 32, "mxfp8_quantize_sr");
@@ -257,6 +259,7 @@ nvfp4moe_status rht32_quantize(const uint16_t *x, int64_t rows, int64_t cols, in
          "rht32_quantize: only the ROWMAJOR scale layout is implemented");
     NEED(cols % 32 == 0 && ld % 8 == 0 && ld >= cols, NVFP4MOE_ERR_SHAPE,
          "rht32_quantize: cols %% 32 == 0, ld %% 8 == 0, ld >= cols required");
+    NEED(rows * (cols / 32) < (1LL << 31), NVFP4MOE_ERR_SHAPE, "rht32_quantize: tensor too large");
     if (rows * cols) {
         NEED_PTR(x);
         NEED_PTR(codes);

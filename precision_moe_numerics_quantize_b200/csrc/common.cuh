@@ -165,23 +165,34 @@ NV_DEV float scale_pow2(float v, int k) {
     return v * exp2i(nk);
 }
 
-// E4M3 code of v with stochastic rounding driven by the 32-bit word r:
-// E4M3 spacing q = 2^(max(floor(log2|v|), -6) - 3); with lo = floor(|v|/q)*q,
-// round up iff (r >> 8) * 2^-24 < (|v| - lo) / q. |v| <= 448 is assumed.
-NV_DEV uint32_t e4m3_encode_sr(float v, uint32_t r) {
-    float a = fabsf(v);
-    uint32_t u = __float_as_uint(a);
-    int e = (int)((u >> 23) & 0xFF) - 127;
-    if (e < -6) e = -6;
-    float inv_q = exp2i(3 - e);       // 1/q, exact
-    float m = a * inv_q;              // exact: |v| has at most 24 significant bits
-    float lo = floorf(m);
-    float frac = m - lo;              // exact
-    float rr = (float)(r >> 8) * 5.9604644775390625e-08f;  // r * 2^-24, exact
-    float mag = (rr < frac) ? lo + 1.0f : lo;
-    float res = mag * exp2i(e - 3);   // exact
-    return e4m3_encode_pos(res) | ((__float_as_uint(v) >> 24) & 0x80u);
+// v rounded stochastically onto the E4M3 grid (sign kept), as an fp32 value,
+// driven by the 32-bit word r: with lo <= |v| <= hi the neighbouring E4M3
+// values, round up iff (r >> 8) * 2^-24 < (|v| - lo) / (hi - lo). |v| <= 448.
+// E4M3 normal range (|v| >= 2^-6): E4M3 keeps 3 of the 23 fp32 mantissa bits,
+// the fraction is the 20 dropped bits / 2^20, and the test is the integer
+// comparison (r >> 8) < dropped << 4; a carry out of the kept mantissa moves to
+// the next binade, which is the correct neighbour. Below 2^-6 the spacing is
+// 2^-9 and the fraction is taken in exact fp32 arithmetic.
+NV_DEV float e4m3_sr_value(float v, uint32_t r) {
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t a = u & 0x7FFFFFFFu;
+    const uint32_t r24 = r >> 8;
+    if (a >= 0x3C800000u) {
+        const uint32_t low = a & 0xFFFFFu;
+        uint32_t kept = a & ~0xFFFFFu;
+        if (r24 < (low << 4)) kept += 0x100000u;
+        return __uint_as_float(kept | (u & 0x80000000u));
+    }
+    const float m = __uint_as_float(a) * 512.0f;  // exact
+    const float lo = floorf(m);
+    const float frac = m - lo;                    // exact
+    const float rr = (float)r24 * 5.9604644775390625e-08f;
+    const float mag = (rr < frac) ? lo + 1.0f : lo;
+    return copysignf(mag * 0.001953125f, v);      // exact
 }
+
+// E4M3 code of v with stochastic rounding (see e4m3_sr_value).
+NV_DEV uint32_t e4m3_encode_sr(float v, uint32_t r) { return e4m3_encode(e4m3_sr_value(v, r)); }
 
 // ---------------------------------------------------------------------------
 // NVFP4 block of 16: per-tensor S_enc, block scale s = E4M3((amax_b / 6) * S_enc),
@@ -209,6 +220,32 @@ NV_DEV uint32_t nvfp4_block16(const float *v, float S_enc, uint32_t &w0, uint32_
                    __fmul_rn(v[11], enc), __fmul_rn(v[12], enc), __fmul_rn(v[13], enc),
                    __fmul_rn(v[14], enc), __fmul_rn(v[15], enc));
     return sc;
+}
+
+// Same block quantization with the per-tensor table enc_tab[c] = S_enc / e4m3(c)
+// (enc_tab[0] = 0), built once per CTA with the same correctly rounded division,
+// and the scale code from the hardware conversion: identical results.
+NV_DEV uint32_t nvfp4_block16_tab(const float *v, float S_enc, const float *enc_tab, uint32_t &w0,
+                                  uint32_t &w1) {
+    float amax_b = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+    const float t = __fmul_rn(__fdiv_rn(amax_b, 6.0f), S_enc);
+    const uint32_t sc = e4m3x2_hw(t, 0.0f) & 0xFFu;
+    const float enc = enc_tab[sc];
+    w0 = e2m1x8_hw(__fmul_rn(v[0], enc), __fmul_rn(v[1], enc), __fmul_rn(v[2], enc),
+                   __fmul_rn(v[3], enc), __fmul_rn(v[4], enc), __fmul_rn(v[5], enc),
+                   __fmul_rn(v[6], enc), __fmul_rn(v[7], enc));
+    w1 = e2m1x8_hw(__fmul_rn(v[8], enc), __fmul_rn(v[9], enc), __fmul_rn(v[10], enc),
+                   __fmul_rn(v[11], enc), __fmul_rn(v[12], enc), __fmul_rn(v[13], enc),
+                   __fmul_rn(v[14], enc), __fmul_rn(v[15], enc));
+    return sc;
+}
+
+// enc_tab for one tensor scale, filled by the threads of a CTA (then sync).
+NV_DEV void fill_enc_table(float *enc_tab, float S_enc) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x)
+        enc_tab[c] = (c == 0 || c == 127) ? 0.0f : __fdiv_rn(S_enc, e4m3_decode_pos((uint32_t)c));
 }
 
 NV_DEV void unpack_bf16x8(uint4 q, float *f) {

@@ -20,17 +20,34 @@ __device__ int32_t g_device_error = 0;
 __global__ void __launch_bounds__(256) amax_bf16_kernel(const uint16_t *__restrict__ x,
                                                         int64_t rows, int64_t cols, int64_t ld,
                                                         float *__restrict__ amax) {
-    const int64_t vpr = cols / 8;  // 16-byte vectors per row
-    const int64_t nvec = rows * vpr;
     float m = 0.0f;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t r = i / vpr, c = i - r * vpr;
-        uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + r * ld) + c);
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
-                           fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))),
-                           fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    if (ld == cols) {
+        // contiguous: one flat run of 16-byte vectors, two loads in flight per step
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+        const int64_t nvec = rows * cols / 8;
+        for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec; i += 2 * stride) {
+            const uint4 v = __ldg(xv + i);
+            const uint4 w = (i + stride < nvec) ? __ldg(xv + i + stride) : make_uint4(0, 0, 0, 0);
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
+                               fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))),
+                               fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(w.x)), fabsf(bf16_hi(w.x))),
+                               fmaxf(fabsf(bf16_lo(w.y)), fabsf(bf16_hi(w.y)))));
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(w.z)), fabsf(bf16_hi(w.z))),
+                               fmaxf(fabsf(bf16_lo(w.w)), fabsf(bf16_hi(w.w)))));
+        }
+    } else {
+        const int64_t vpr = cols / 8;  // 16-byte vectors per row
+        for (int64_t r = blockIdx.y; r < rows; r += gridDim.y)
+            for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < vpr; c += stride) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + r * ld) + c);
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
+                                   fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))),
+                                   fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+            }
     }
     m = warp_max(m);
     __shared__ float red[8];
@@ -67,27 +84,51 @@ NV_DEV uint32_t nvfp4_quant64(const uint16_t *__restrict__ p, float S_enc, uint4
     return scw;
 }
 
+// Same with the per-tensor encode table; all eight 16-byte loads issued first.
+NV_DEV uint32_t nvfp4_quant64_tab(const uint16_t *__restrict__ p, float S_enc, const float *enc_tab,
+                                  uint4 &c0, uint4 &c1) {
+    const uint4 *pv = reinterpret_cast<const uint4 *>(p);
+    uint4 raw[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) raw[j] = __ldg(pv + j);
+    uint32_t scw = 0;
+    uint32_t w[8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        float v[16];
+        unpack8(raw[2 * b], v);
+        unpack8(raw[2 * b + 1], v + 8);
+        uint32_t sc = nvfp4_block16_tab(v, S_enc, enc_tab, w[2 * b], w[2 * b + 1]);
+        scw |= sc << (8 * b);
+    }
+    c0 = make_uint4(w[0], w[1], w[2], w[3]);
+    c1 = make_uint4(w[4], w[5], w[6], w[7]);
+    return scw;
+}
+
 __global__ void __launch_bounds__(256) nvfp4_quant_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     const float *__restrict__ amax_p, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
     float *__restrict__ ts_out, int layout) {
+    __shared__ float enc_tab[128];
     const float amax = *amax_p;
     const float S_enc = nvfp4_senc(amax);
-    const int64_t G = cols / 64;
-    const int64_t n = rows * G;
+    fill_enc_table(enc_tab, S_enc);
+    __syncthreads();
+    const uint32_t G = (uint32_t)(cols / 64);
+    const uint32_t n = (uint32_t)(rows * G);  // < 2^31 (checked by the caller)
     if (ts_out && blockIdx.x == 0 && threadIdx.x == 0) *ts_out = nvfp4_ts(amax);
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t r = i / G, g = i - r * G;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t r = i / G, g = i - r * G;
         uint4 c0, c1;
-        uint32_t scw = nvfp4_quant64(x + r * ld + g * 64, S_enc, c0, c1);
-        uint4 *co = reinterpret_cast<uint4 *>(codes + r * (cols / 2) + g * 32);
+        const uint32_t scw = nvfp4_quant64_tab(x + (int64_t)r * ld + g * 64, S_enc, enc_tab, c0, c1);
+        uint4 *co = reinterpret_cast<uint4 *>(codes + (int64_t)i * 32);
         co[0] = c0;
         co[1] = c1;
         if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
-            *reinterpret_cast<uint32_t *>(scales + r * (cols / 16) + g * 4) = scw;
+            *reinterpret_cast<uint32_t *>(scales + (int64_t)i * 4) = scw;
         else
-            *reinterpret_cast<uint32_t *>(scales + mma_sf_offset(r, g * 4, cols / 16)) = scw;
+            *reinterpret_cast<uint32_t *>(scales + mma_sf_offset(r, g * 4, G * 4)) = scw;
     }
 }
 
@@ -133,22 +174,21 @@ NV_DEV uint32_t mx_block32(const float (&v)[32], uint64_t seed, uint64_t offset,
     float amax_b = 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
-    int k = mx_scale_exp(amax_b);
+    const int k = mx_scale_exp(amax_b);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        uint32_t word = 0;
+        float s0 = scale_pow2(v[4 * q], k), s1 = scale_pow2(v[4 * q + 1], k);
+        float s2 = scale_pow2(v[4 * q + 2], k), s3 = scale_pow2(v[4 * q + 3], k);
         if (SR) {
-            // idx0 is a multiple of 4 here (cols % 32 == 0): one Philox call per 4 elements
-            u32x4 r = philox_block(seed, offset, (idx0 >> 2) + q);
-            uint32_t rs[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                word |= e4m3_encode_sr(scale_pow2(v[4 * q + j], k), rs[j]) << (8 * j);
-        } else {
-            word = e4m3x2_hw(scale_pow2(v[4 * q], k), scale_pow2(v[4 * q + 1], k)) |
-                   (e4m3x2_hw(scale_pow2(v[4 * q + 2], k), scale_pow2(v[4 * q + 3], k)) << 16);
+            // idx0 is a multiple of 4 (cols % 32 == 0): one Philox call per 4 elements
+            const u32x4 r = philox_block(seed, offset, (idx0 >> 2) + q);
+            s0 = e4m3_sr_value(s0, r.x);
+            s1 = e4m3_sr_value(s1, r.y);
+            s2 = e4m3_sr_value(s2, r.z);
+            s3 = e4m3_sr_value(s3, r.w);
         }
-        w[q] = word;
+        // on-grid values (SR) convert exactly; otherwise this is the RNE encode
+        w[q] = e4m3x2_hw(s0, s1) | (e4m3x2_hw(s2, s3) << 16);
     }
     return (uint32_t)(k + 127);
 }
@@ -157,22 +197,24 @@ template <bool SR>
 __global__ void __launch_bounds__(256) mxfp8_rows_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
     uint64_t offset, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int layout) {
-    const int64_t G = cols / 32;  // blocks per row
-    const int64_t n = rows * G;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t r = i / G, b = i - r * G;
-        const uint4 *pv = reinterpret_cast<const uint4 *>(x + r * ld + b * 32);
+    const uint32_t G = (uint32_t)(cols / 32);  // blocks per row
+    const uint32_t n = (uint32_t)(rows * G);
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t r = i / G, b = i - r * G;
+        const uint4 *pv = reinterpret_cast<const uint4 *>(x + (int64_t)r * ld + b * 32);
+        uint4 raw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) raw[j] = __ldg(pv + j);
         float v[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) unpack8(__ldg(pv + j), v + 8 * j);
+        for (int j = 0; j < 4; ++j) unpack8(raw[j], v + 8 * j);
         uint32_t w[8];
-        uint32_t sc = mx_block32<SR>(v, seed, offset, (uint64_t)(r * cols + b * 32), w);
-        uint4 *co = reinterpret_cast<uint4 *>(codes + r * cols + b * 32);
+        const uint32_t sc = mx_block32<SR>(v, seed, offset, (uint64_t)r * cols + b * 32, w);
+        uint4 *co = reinterpret_cast<uint4 *>(codes + (int64_t)i * 32);
         co[0] = make_uint4(w[0], w[1], w[2], w[3]);
         co[1] = make_uint4(w[4], w[5], w[6], w[7]);
         if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
-            scales[r * G + b] = (uint8_t)sc;
+            scales[i] = (uint8_t)sc;
         else
             scales[mma_sf_offset(r, b, G)] = (uint8_t)sc;
     }
@@ -234,17 +276,17 @@ __global__ void __launch_bounds__(256) mxfp8_cols_kernel(
                 const float v0 = scale_pow2(bf16_lo(pr.x), k0), v1 = scale_pow2(bf16_hi(pr.x), k1);
                 const float v2 = scale_pow2(bf16_lo(pr.y), k2), v3 = scale_pow2(bf16_hi(pr.y), k3);
                 uint32_t e0, e1, e2, e3;
+                float w0v = v0, w1v = v1, w2v = v2, w3v = v3;
                 if (SR) {
                     // elements (rbase + i, c .. c + 3): row-major index multiple of 4
                     const u32x4 r4 = philox_block(seed, offset, (uint64_t)((rbase + i) * cols + c) >> 2);
-                    e0 = e4m3_encode_sr(v0, r4.x);
-                    e1 = e4m3_encode_sr(v1, r4.y);
-                    e2 = e4m3_encode_sr(v2, r4.z);
-                    e3 = e4m3_encode_sr(v3, r4.w);
-                } else {
-                    const uint32_t p01 = e4m3x2_hw(v0, v1), p23 = e4m3x2_hw(v2, v3);
-                    e0 = p01 & 0xFFu; e1 = p01 >> 8; e2 = p23 & 0xFFu; e3 = p23 >> 8;
+                    w0v = e4m3_sr_value(v0, r4.x);
+                    w1v = e4m3_sr_value(v1, r4.y);
+                    w2v = e4m3_sr_value(v2, r4.z);
+                    w3v = e4m3_sr_value(v3, r4.w);
                 }
+                const uint32_t p01 = e4m3x2_hw(w0v, w1v), p23 = e4m3x2_hw(w2v, w3v);
+                e0 = p01 & 0xFFu; e1 = p01 >> 8; e2 = p23 & 0xFFu; e3 = p23 >> 8;
                 a0 |= e0 << (8 * j);
                 a1 |= e1 << (8 * j);
                 a2 |= e2 << (8 * j);
@@ -331,13 +373,13 @@ __global__ void __launch_bounds__(256) rht32_amax_kernel(const uint16_t *__restr
                                                          uint64_t sign_seed,
                                                          float *__restrict__ amax) {
     const uint32_t signs = rht_signs_dev(sign_seed);
-    const int64_t G = cols / 32;
+    const uint32_t G = (uint32_t)(cols / 32);
+    const uint32_t n = (uint32_t)(rows * G);
     float m = 0.0f;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t r = i / G, b = i - r * G;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t r = i / G, b = i - r * G;
         float v[32];
-        rht32_fwd(x + r * ld + b * 32, signs, v);
+        rht32_fwd(x + (int64_t)r * ld + b * 32, signs, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
     }
@@ -356,33 +398,35 @@ __global__ void __launch_bounds__(256) rht32_quant_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t sign_seed,
     int fmt, const float *__restrict__ amax_p, uint8_t *__restrict__ codes,
     uint8_t *__restrict__ scales, float *__restrict__ ts_out) {
+    __shared__ float enc_tab[128];
     const uint32_t signs = rht_signs_dev(sign_seed);
-    const int64_t G = cols / 32;
+    const uint32_t G = (uint32_t)(cols / 32);
+    const uint32_t n = (uint32_t)(rows * G);
     float S_enc = 1.0f;
     if (fmt == NVFP4MOE_FMT_NVFP4) {
-        float amax = *amax_p;
+        const float amax = *amax_p;
         S_enc = nvfp4_senc(amax);
+        fill_enc_table(enc_tab, S_enc);
         if (ts_out && blockIdx.x == 0 && threadIdx.x == 0) *ts_out = nvfp4_ts(amax);
     }
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t r = i / G, b = i - r * G;
+    __syncthreads();
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t r = i / G, b = i - r * G;
         float v[32];
-        rht32_fwd(x + r * ld + b * 32, signs, v);
+        rht32_fwd(x + (int64_t)r * ld + b * 32, signs, v);
         if (fmt == NVFP4MOE_FMT_NVFP4) {
             uint32_t w0, w1, w2, w3;
-            uint32_t s0 = nvfp4_block16(v, S_enc, w0, w1);
-            uint32_t s1 = nvfp4_block16(v + 16, S_enc, w2, w3);
-            *reinterpret_cast<uint4 *>(codes + r * (cols / 2) + b * 16) = make_uint4(w0, w1, w2, w3);
-            *reinterpret_cast<uint16_t *>(scales + r * (cols / 16) + b * 2) =
-                (uint16_t)(s0 | (s1 << 8));
+            const uint32_t s0 = nvfp4_block16_tab(v, S_enc, enc_tab, w0, w1);
+            const uint32_t s1 = nvfp4_block16_tab(v + 16, S_enc, enc_tab, w2, w3);
+            *reinterpret_cast<uint4 *>(codes + (int64_t)i * 16) = make_uint4(w0, w1, w2, w3);
+            *reinterpret_cast<uint16_t *>(scales + (int64_t)i * 2) = (uint16_t)(s0 | (s1 << 8));
         } else {
             uint32_t w[8];
-            uint32_t sc = mx_block32<false>(v, 0, 0, 0, w);
-            uint4 *co = reinterpret_cast<uint4 *>(codes + r * cols + b * 32);
+            const uint32_t sc = mx_block32<false>(v, 0, 0, 0, w);
+            uint4 *co = reinterpret_cast<uint4 *>(codes + (int64_t)i * 32);
             co[0] = make_uint4(w[0], w[1], w[2], w[3]);
             co[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            scales[r * G + b] = (uint8_t)sc;
+            scales[i] = (uint8_t)sc;
         }
     }
 }
@@ -446,7 +490,13 @@ cudaError_t launch_amax_bf16(const uint16_t *x, int64_t rows, int64_t cols, int6
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
     if (e != cudaSuccess) return e;
     if (rows * cols == 0) return cudaSuccess;
-    amax_bf16_kernel<<<grid_for(rows * (cols / 8)), 256, 0, s>>>(x, rows, cols, ld, amax);
+    if (ld == cols) {
+        amax_bf16_kernel<<<grid_for(rows * cols / 16), 256, 0, s>>>(x, rows, cols, ld, amax);
+    } else {
+        const int64_t vpr = cols / 8;
+        dim3 grid((unsigned)((vpr + 255) / 256), (unsigned)(rows < 1024 ? rows : 1024));
+        amax_bf16_kernel<<<grid, 256, 0, s>>>(x, rows, cols, ld, amax);
+    }
     return cudaGetLastError();
 }
 

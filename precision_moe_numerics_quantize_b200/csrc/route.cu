@@ -206,21 +206,27 @@ __global__ void __launch_bounds__(256) dispatch_quant_kernel(
     const float *__restrict__ amax_p, const int32_t *__restrict__ pos,
     uint8_t *__restrict__ xq, uint8_t *__restrict__ xq_sc, float *__restrict__ x_ts,
     int write_ts) {
+    __shared__ float enc_tab[128];
     const float amax = *amax_p;
     const float S_enc = nvfp4_senc(amax);
+    fill_enc_table(enc_tab, S_enc);
+    __syncthreads();
     if (write_ts && blockIdx.x == 0 && threadIdx.x == 0) *x_ts = nvfp4_ts(amax);
     const int64_t G = d / 64;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < T * G;
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t t = i / G, g = i - t * G;
         const uint4 *pv = reinterpret_cast<const uint4 *>(x + t * d + g * 64);
+        uint4 raw[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) raw[j] = __ldg(pv + j);
         uint32_t w[8], scw = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
             float v[16];
-            unpack_bf16x8(__ldg(pv + 2 * b), v);
-            unpack_bf16x8(__ldg(pv + 2 * b + 1), v + 8);
-            scw |= nvfp4_block16(v, S_enc, w[2 * b], w[2 * b + 1]) << (8 * b);
+            unpack_bf16x8(raw[2 * b], v);
+            unpack_bf16x8(raw[2 * b + 1], v + 8);
+            scw |= nvfp4_block16_tab(v, S_enc, enc_tab, w[2 * b], w[2 * b + 1]) << (8 * b);
         }
         const uint4 c0 = make_uint4(w[0], w[1], w[2], w[3]);
         const uint4 c1 = make_uint4(w[4], w[5], w[6], w[7]);
