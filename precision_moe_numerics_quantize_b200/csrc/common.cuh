@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "../../include/nvfp4moe.h"
@@ -30,6 +31,9 @@ enum WaitId : int32_t {
     WAIT_GEMM_ACC_FULL = 3,
     WAIT_GEMM_ACC_EMPTY = 4,
     WAIT_GEMM_DRAIN = 5,
+    WAIT_GEMM_SF_SLOT = 6,
+    WAIT_GEMM_SF_FULL = 7,
+    WAIT_GEMM_SF_READY = 8,
 };
 
 // ---------------------------------------------------------------------------
@@ -44,6 +48,12 @@ NV_DEV uint32_t f32_to_bf16_bits(float f) {
     if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return 0x7FC0u;
     u += 0x7FFFu + ((u >> 16) & 1u);
     return u >> 16;
+}
+
+// Two floats to a bf16 pair, round to nearest even (lo in bits 0..15).
+NV_DEV uint32_t bf16x2_rn(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
 }
 
 NV_DEV float warp_max(float v) {
@@ -365,22 +375,84 @@ NV_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
         : "memory");
 }
 
+// Per-thread asynchronous copies global -> shared (cp.async), with their
+// completion counted on an mbarrier: the arrival is made when all of this
+// thread's earlier cp.async copies have landed, and does not increment the
+// barrier's pending count (it was initialised with one count per thread).
+NV_DEV void cp_async_16(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+NV_DEV void cp_async_4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+NV_DEV void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 NV_DEV void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// --- tcgen05 ---------------------------------------------------------------
-NV_DEV void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+// --- clusters ----------------------------------------------------------------
+NV_DEV uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address in the shared::cluster window of the same variable in CTA `rank`.
+NV_DEV uint32_t cluster_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+// Arrive on an mbarrier of any CTA of the cluster without release semantics:
+// for hand-offs of TMEM whose reads or writes this thread has already waited
+// for (tcgen05.wait::ld / ::st, then tcgen05.fence::before_thread_sync). A
+// cluster-scope release would also wait for every generic store of the thread
+// to become visible, which costs about a thousand cycles while the SM streams
+// epilogue stores.
+NV_DEV void mbar_arrive_cluster_relaxed(uint32_t cbar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar)
+                 : "memory");
+}
+// All threads of every CTA of the cluster.
+NV_DEV void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA tiled loads issued by either CTA of a pair into its own shared memory,
+// the completed bytes counted on an mbarrier given by its shared::cluster
+// address (the pair's first CTA holds it).
+NV_DEV void tma_load_2d_pair(void *dst, const CUtensorMap *map, int32_t x, int32_t y,
+                             uint32_t cbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(cbar)
+        : "memory");
+}
+NV_DEV void tma_load_5d_pair(void *dst, const CUtensorMap *map, int32_t c0, int32_t c1, int32_t c2,
+                             int32_t c3, int32_t c4, uint32_t cbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+        "r"(cbar)
+        : "memory");
+}
+
+// --- tcgen05 (CTA pairs: every tcgen05 op of a kernel uses one cta_group) ----
+NV_DEV void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(dst_smem)),
                  "r"(ncols)
                  : "memory");
 }
-NV_DEV void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+NV_DEV void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
 }
-NV_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+NV_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                  : "memory");
 }
 NV_DEV void tc_fence_before() {
@@ -389,35 +461,38 @@ NV_DEV void tc_fence_before() {
 NV_DEV void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// Arrive on an mbarrier once every previously issued tcgen05 op of this thread completes.
-NV_DEV void tc_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-// Copy a 32-row x 128-bit block from shared memory into TMEM, replicated to
-// all four 32-lane sub-partitions.
-NV_DEV void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+// Arrive on an mbarrier (shared::cluster address, either CTA of the pair) once
+// every tcgen05 op issued so far by this thread has completed.
+NV_DEV void tc_commit_pair(uint32_t cbar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     cbar)
                  : "memory");
 }
-NV_DEV void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+// The same, arriving on the mbarrier at this shared::cta offset in every CTA
+// of `cta_mask` (one tensor-core commit, no memory load involved).
+NV_DEV void tc_commit_pair_mc(uint32_t cbar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+        "[%0], %1;" ::"r"(cbar),
+        "h"(cta_mask)
+        : "memory");
+}
+NV_DEV void tc_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
         "[%6], p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");
 }
-NV_DEV void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+NV_DEV void tc_mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], "
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], "
         "p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");

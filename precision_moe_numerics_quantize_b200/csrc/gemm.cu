@@ -1,40 +1,79 @@
-// Grouped block-scaled GEMM on the sm_100a tensor cores (tcgen05).
+// Grouped block-scaled GEMM on the sm_100a tensor cores, one CTA pair per
+// tile (tcgen05.mma.cta_group::2).
 //
-// One persistent CTA per SM walks a list of 128 x 256 output tiles. Tiles are
-// enumerated group by group (an expert is a group), N-tile major and M-tile
-// minor, so neighbouring CTAs share the weight tile through L2. The tile list
-// is derived on the device from the group offsets: no host synchronisation.
+// Every product in this file has the form
+//     out[x, w] = alpha_g * sum_k X[x, k] * W[w, k]
+// with X the token-side operand (activations or gradients: rows grouped by
+// expert, or one row set whose contraction columns are split by group) and W
+// the weights of group g. The MMA's M side is W: a cluster of two CTAs on two
+// SMs computes a tile of 256 W rows x n X rows. Each CTA stages 128 W rows and
+// n/2 X rows per k-block; the MMA reads the operands from both CTAs' shared
+// memory, and each CTA's TMEM receives the fp32 accumulator of its 128 W rows
+// over all n X rows. A group's (128-padded) X rows are cut into the fewest
+// tiles of at most 192 rows, of equal size rounded up to 64: a 384-row expert
+// becomes 2 x 192, not 256 + 128. A pair MMA of N = 192 runs at the full
+// tensor rate, one of N = 128 is limited by how fast one thread can issue it.
 //
-// Roles (448 threads, 14 warps):
-//   warp 0       TMA producer: per 128-byte K stage, the A tile (128 rows),
-//                the B tile (two 128-row halves) with 128-byte swizzle, and
-//                the block scales (stored in the MMA chunk layout) with plain
-//                bulk copies. STAGES-deep mbarrier ring.
-//   warps 2..5   scale warps, one per TMEM lane quarter: they move each stage's
-//                scales from shared memory into a TMEM ring with tcgen05.st,
-//                in the replicated layout the block-scaled MMA reads (lane r of
-//                every quarter holds the scales of rows r, r+32, r+64, ...).
-//                Doing this with thread stores rather than tcgen05.cp keeps the
-//                tensor pipe for MMAs only: a tcgen05.cp occupies the in-order
-//                tensor pipe about as long as an MMA.
-//   warp 1       MMA issuer (one thread): four block-scaled MMAs per stage
-//                (kind::mxf4nvf4 block16 for NVFP4, kind::mxf8f6f4 with E8M0
-//                scales for MXFP8) into the TMEM accumulator; tcgen05.commit
-//                frees the stage and finally signals the accumulator.
-//   warps 6..13  epilogue: tcgen05.ld of the fp32 accumulator (warp w reads
-//                lanes 32*(w%4)..+31, two warps per quarter split the columns),
-//                released back to the MMA warp as soon as it is in registers;
-//                then SwiGLU with a fused per-group amax, or a bf16 / fp32 store.
-// TMEM: columns [0, 256) accumulator, [256, 512) scale ring, 64 columns per
-// stage: B scales of MMA kb at +8kb .. +8kb+7 (every lane quarter holds all 256
-// B rows); A scales of MMA kb at the 4-column group +32+4kb (lane quarter q,
-// which computes rows 32q..32q+31, reads column +32+4kb+q, so each quarter
-// writes only that one column). Scale addresses given to the MMA and the
-// column of every multi-column tcgen05.st stay 4-column aligned.
+// A pipeline stage is 256 bytes of K (two 128-byte k-blocks, eight MMAs): the
+// MMA-issuing thread pays one barrier wait, one fence and one commit per stage.
+// Every barrier operation costs a few hundred cycles while the tensor cores
+// and TMA keep shared memory busy, so each role does as few per stage as the
+// protocol allows.
 //
-// Every wait is bounded (about 2 s); a wait that runs out records its id in
-// the device error word, raises a CTA-wide abort flag and the kernel winds
-// down, releasing TMEM.
+// Roles (448 threads, 14 warps, in both CTAs of the pair):
+//   warp 0       TMA producer: this CTA's W and X halves (128-byte swizzle),
+//                completion counted on the first CTA's `full` barrier, and
+//                the X block scales of the stage (plain bulk copies of the one
+//                or two 128-row chunk rows) into this CTA: counted on `full`
+//                in the first CTA, on its own `sf_loaded` in the other.
+//   warps 2..5   scale warps, one per TMEM lane quarter (SCALE_SETS sets of
+//                four can take turns by stage). Each lane reads the stage's X
+//                scale words from shared memory and the W scale words of its
+//                own TMEM lane, loaded from L2 one stage ahead, and writes them
+//                with tcgen05.st into the stage's scale slot in this CTA's
+//                TMEM, in the layout the block-scaled MMA reads (the X scales
+//                of all n rows in every lane quarter; the W scale word of lane
+//                32q + l in column q of a 4-column group). One scale slot per
+//                shared-memory stage: the producer only loads a stage once the
+//                MMAs of the stage that last used its slot are done, so the
+//                one wait for the stage's bytes also frees the slot (and, in
+//                the first CTA, vouches for the operands); one arrival per
+//                stage on the first CTA's sf_full follows. Thread stores keep
+//                the in-order tensor pipe for MMAs only.
+//   warp 1       first CTA only: the MMA issuer (one thread), eight
+//                block-scaled MMAs per stage (kind::mxf4nvf4 block16 for
+//                NVFP4, kind::mxf8f6f4 with E8M0 scales for MXFP8) after one
+//                wait on sf_full; one commit multicast to both CTAs' `empty`
+//                barriers per stage and, after a tile's last stage, to both
+//                `acc_full` barriers.
+//   warps 6..13  epilogue: two warps per lane quarter, n/2 accumulator
+//                columns each, read with tcgen05.ld in two round trips of at
+//                most 64 columns and packed to bf16 pairs (SwiGLU: finished to
+//                h first), so that the whole share fits in registers; the
+//                accumulator goes back to the MMA warp (arrival on the first
+//                CTA's acc_empty) as soon as the last columns are in
+//                registers, and the stores follow. Lane =
+//                output column, register = output row, so every store
+//                instruction of a warp writes one contiguous run of an output
+//                row.
+// SwiGLU (first GEMM of the expert FFN): W = [gate; up]. The W box of a CTA
+// holds, per lane quarter, 16 gate rows followed by the 16 up rows of the same
+// h columns (one 5-D TMA box), so lanes l and l ^ 16 of a warp hold g and u of
+// one h column and trade half their values with one shuffle each.
+// TMEM: columns [0, 192) accumulator, then one scale slot of 96 columns per
+// shared-memory stage, 48 per k-block j: X scales of MMA kb at +48j+8kb (8
+// columns = 256 rows), W scales of MMA kb at +48j+32+4kb (column q is read by
+// lane quarter q). Every multi-column tcgen05.st and every scale address given
+// to the MMA is 4-column aligned.
+//
+// Arrivals between the CTAs of a pair are relaxed: what they hand over is
+// TMEM, ordered by tcgen05.wait and the tcgen05 fences; a cluster-scope
+// release would also wait for the epilogue's global stores.
+//
+// Every wait is bounded (about 2 s): a wait that runs out records its id in
+// the device error word and raises this CTA's abort flag; the CTA winds down
+// and the other CTA of the pair then runs out on its own waits. Both CTAs meet
+// at a final cluster barrier before TMEM is released.
 #include "common.cuh"
 #include "quant.cuh"
 
@@ -44,104 +83,140 @@ namespace nvfp4moe {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, KBYTES = 128, STAGES = 4;
-constexpr int A_STAGE = BM * KBYTES;   // 16 KB
-constexpr int B_STAGE = BN * KBYTES;   // 32 KB
-constexpr int SFA_STAGE = 2048, SFB_STAGE = 4096;
-constexpr int NUM_THREADS = 448;
+constexpr int STAGES = 3;                // shared-memory stages of 2 k-blocks
+constexpr int MAX_N = 192;               // X rows per tile
+constexpr int W_KBLK = 128 * 128;        // one k-block (128 bytes of K) of 128 W rows
+constexpr int X_KBLK = (MAX_N / 2) * 128;  // one k-block of up to 96 X rows
+constexpr int W_STAGE = 2 * W_KBLK;
+constexpr int X_STAGE = 2 * X_KBLK;
+// X block scales of a stage: two 128-row chunk rows x 8 chunks of 512 bytes
+// (NVFP4: 4 chunks per k-block; MXFP8: 1)
+constexpr int SFX_CHUNKS = 8, SFX_STAGE = 2 * SFX_CHUNKS * 512;
+// scale warps come in SCALE_SETS sets of four taking turns by stage; the
+// epilogue's two warps per lane quarter follow them
+constexpr int SCALE_SETS = 1;
+constexpr int SCALE_WARP0 = 2, EPI_WARP0 = SCALE_WARP0 + 4 * SCALE_SETS;
+constexpr int NUM_THREADS = 32 * (EPI_WARP0 + 8);
 constexpr int MAX_GROUPS = 1024;
-constexpr uint32_t TMEM_COLS = 512, TMEM_SF = 256, SF_SLOT_COLS = 64;
+constexpr uint32_t TMEM_COLS = 512, TMEM_SF = MAX_N, SF_KB_COLS = 48, SF_SLOT_COLS = 96;
 
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
-constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
-constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-// barriers: full[S] (operands), sf_loaded[S] (scales in smem), sf_full[S]
-// (scales in TMEM), empty[S], acc_full, acc_empty
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int OFF_MISC = OFF_BAR + 8 * (4 * STAGES + 2);  // tmem base, abort flag
-constexpr int OFF_PREFIX = OFF_MISC + 16;
-constexpr int SMEM_BYTES = OFF_PREFIX + 4 * (MAX_GROUPS + 1);
+constexpr int OFF_W = 0;
+constexpr int OFF_X = OFF_W + STAGES * W_STAGE;
+constexpr int OFF_SFX = OFF_X + STAGES * X_STAGE;
+// barriers: full[SETS S], empty[S], sf_full[S], sf_loaded[SETS S], acc_full,
+// acc_empty. `full` and `sf_loaded` are waited on by the scale-warp set that
+// handles the stage: stage i uses barrier stage_bar(i) = (i % SETS) S +
+// (i / SETS) % S, so every barrier is waited on by one set, in order, and a
+// parity wait can never alias a phase two uses ahead.
+constexpr int OFF_BAR = OFF_SFX + STAGES * SFX_STAGE;
+constexpr int NUM_BARS = (2 * SCALE_SETS + 2) * STAGES + 2;
+constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;               // tmem base, abort flag
+constexpr int OFF_GTAB = OFF_MISC + 16;  // per-group tile table (int4), one sentinel
+constexpr int SMEM_BYTES = OFF_GTAB + 16 * (MAX_GROUPS + 1);
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
+static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+static_assert(X_KBLK % 1024 == 0, "k-block areas stay 1024-byte aligned");
+static_assert(TMEM_SF + STAGES * SF_SLOT_COLS <= TMEM_COLS, "TMEM columns");
+
+constexpr uint32_t FULL_COUNT = 1;        // the first CTA's producer
+constexpr uint32_t SF_FULL_COUNT = 8;     // 4 scale warps x 2 CTAs
+constexpr uint32_t ACC_EMPTY_COUNT = 16;  // 8 epilogue warps x 2 CTAs
+
+__host__ __device__ constexpr uint32_t stage_bar(uint32_t i) {
+    return (i % SCALE_SETS) * STAGES + (i / SCALE_SETS) % STAGES;
+}
+__host__ __device__ constexpr uint32_t stage_par(uint32_t i) { return ((i / SCALE_SETS) / STAGES) & 1u; }
 
 struct Params {
     int kind, epi, group_axis;
-    const uint8_t *a_sc, *b_sc;
-    const float *a_ts, *b_ts;
-    int32_t a_ts_stride;
+    const uint8_t *w_sc, *x_sc;
+    const float *w_ts, *x_ts;
+    int32_t x_ts_stride;
     const int32_t *group_off;
     int32_t G;
-    int64_t M;             // group K: rows of each output block
-    int64_t N;             // accumulator columns per group (SwiGLU: 2f)
+    int64_t x_rows;        // group K: X rows, the output rows of every group
+    int64_t w_rows_group;  // W rows per group (SwiGLU: 2f); 0 when W is shared
     int64_t f_out;         // SwiGLU: f
     int64_t ldc;           // output row stride (elements)
-    int64_t b_rows_per_group;
-    int64_t a_nkc, b_nkc;  // 512-byte scale chunks per 128-row block
-    int32_t kt_total;      // K stages (group M)
+    int64_t w_nkc, x_nkc;  // 512-byte scale chunks per 128-row block
+    int32_t kt_total;      // 128-byte k-blocks of K (group M)
+    int32_t wtiles;        // 256-row W tiles per group (SwiGLU: f / 128)
     void *c;
     float *amax;
 };
 
 struct Tile {
     int g;
-    int64_t a_row;          // TMA row of A
-    int64_t b_row0, b_row1; // TMA rows of the two B halves
-    int64_t k0;             // first contraction element (group K)
-    int kt;                 // number of K stages
-    int64_t out_row, out_col;
-    int nt, mt;
+    int n;            // X rows of the tile: a multiple of 64, at most MAX_N
+    int mt;           // W tile within the group
+    int kt;           // 128-byte k-blocks of K
+    int64_t x_row;    // first X row (a multiple of 64)
+    int64_t out_row;  // output row of X row x_row
+    int64_t k0;       // first contraction element (group K)
 };
 
-__device__ __forceinline__ int upper_group(const int32_t *prefix, int G, int64_t t) {
-    int lo = 0, hi = G;  // largest g with prefix[g] <= t
-    while (hi - lo > 1) {
-        int mid = (lo + hi) >> 1;
-        if (prefix[mid] <= t) lo = mid; else hi = mid;
-    }
-    return lo;
+// the tiles of `rows` X rows: count, and rows per tile (a multiple of 64)
+__device__ __forceinline__ int32_t x_tiles(int32_t rows) { return (rows + MAX_N - 1) / MAX_N; }
+__device__ __forceinline__ int32_t x_tile_rows(int32_t rows, int32_t ntiles) {
+    return ntiles ? ((rows + ntiles - 1) / ntiles + 63) / 64 * 64 : 0;
 }
 
-__device__ __forceinline__ Tile tile_info(const Params &p, const int32_t *prefix, int64_t t) {
+// Per-group tile table in shared memory, one int4 per group:
+//   x = tiles of the group, y = first X row (group M) or first contraction
+//   element (group K), z = X tiles | rows per X tile << 16,
+//   w = X rows (group M) or 128-byte k-blocks (group K).
+// Every role walks its tiles t = pair, pair + npairs, ... with a cursor
+// (group g, tile within the group) that only moves forward, one table read
+// per group it crosses.
+struct Cursor {
+    int g;
+    int32_t local;
+    int4 e;
+};
+__device__ __forceinline__ void cursor_settle(const int4 *gtab, int G, Cursor &c) {
+    while (c.g < G && c.local >= c.e.x) {
+        c.local -= c.e.x;
+        c.e = gtab[++c.g];
+    }
+}
+__device__ __forceinline__ Cursor cursor_first(const int4 *gtab, int G, int32_t pair) {
+    Cursor c;
+    c.g = 0;
+    c.local = pair;
+    c.e = gtab[0];
+    cursor_settle(gtab, G, c);
+    return c;
+}
+__device__ __forceinline__ void cursor_next(const int4 *gtab, int G, int32_t npairs, Cursor &c) {
+    c.local += npairs;
+    cursor_settle(gtab, G, c);
+}
+
+__device__ __forceinline__ Tile cursor_tile(const Params &p, const Cursor &c) {
     Tile T;
-    const int g = upper_group(prefix, p.G, t);
-    const int64_t local = t - prefix[g];
-    T.g = g;
-    if (p.group_axis == NVFP4MOE_GROUP_M) {
-        const int64_t r0 = p.group_off[g];
-        const int64_t mtiles = ((int64_t)p.group_off[g + 1] - r0) / BM;
-        const int64_t nt = local / mtiles, mt = local - nt * mtiles;
-        T.nt = (int)nt;
-        T.mt = (int)mt;
-        T.a_row = r0 + mt * BM;
-        if (p.epi == EPI_SWIGLU_AMAX) {
-            T.b_row0 = (int64_t)g * p.b_rows_per_group + nt * 128;
-            T.b_row1 = T.b_row0 + p.f_out;
-            T.out_col = nt * 128;
-        } else {
-            T.b_row0 = (int64_t)g * p.b_rows_per_group + nt * BN;
-            T.b_row1 = T.b_row0 + 128;
-            T.out_col = nt * BN;
-        }
+    const int32_t ntiles = c.e.z & 0xFFFF, nb = c.e.z >> 16;
+    const bool gm = p.group_axis == NVFP4MOE_GROUP_M;
+    const int32_t rows = gm ? c.e.w : (int32_t)p.x_rows;
+    const int32_t mt = c.local / ntiles, nt = c.local - mt * ntiles;
+    T.g = c.g;
+    T.mt = mt;
+    T.n = min(nb, rows - nt * nb);
+    if (gm) {
+        T.x_row = (int64_t)c.e.y + (int64_t)nt * nb;
+        T.out_row = T.x_row;
         T.k0 = 0;
         T.kt = p.kt_total;
-        T.out_row = T.a_row;
     } else {
-        const int64_t mtiles = p.M / BM;
-        const int64_t nt = local / mtiles, mt = local - nt * mtiles;
-        T.nt = (int)nt;
-        T.mt = (int)mt;
-        T.a_row = mt * BM;
-        T.b_row0 = nt * BN;
-        T.b_row1 = T.b_row0 + 128;
-        T.k0 = p.group_off[g];
-        T.kt = (int)(((int64_t)p.group_off[g + 1] - T.k0) / 128);
-        T.out_row = (int64_t)g * p.M + T.a_row;
-        T.out_col = nt * BN;
+        T.x_row = (int64_t)nt * nb;
+        T.out_row = (int64_t)c.g * p.x_rows + T.x_row;
+        T.k0 = c.e.y;
+        T.kt = c.e.w;
     }
     return T;
 }
 
-// Bounded wait that also gives up when another role raised the abort flag.
+// Bounded wait that also gives up when another role of this CTA raised the
+// abort flag.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
                                               volatile int32_t *abort_flag, int32_t id) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -157,363 +232,476 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
     }
 }
 
-__device__ __forceinline__ uint32_t idesc_nvf4() {
-    // a/b format E2M1 (1), N >> 3 at bit 17, scale format UE4M3 (0) at bit 23,
-    // M >> 4 at bit 24; K-major A and B; dense.
-    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptors, M = 256 (two CTAs), N = n, K-major A and B, dense.
+__device__ __forceinline__ uint32_t idesc_nvf4(int n) {
+    // a/b format E2M1 (1) at bits 7 and 10, N >> 3 at bit 17, scale format
+    // UE4M3 (0) at bit 23, M >> 4 at bit 24
+    return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (16u << 24);
 }
-__device__ __forceinline__ uint32_t idesc_mxf8(uint32_t sf_id) {
+__device__ __forceinline__ uint32_t idesc_mxf8(int n, uint32_t sf_id) {
     // a/b format E4M3 (0), scale format UE8M0 (1) at bit 23, scale-factor ids
-    // (byte of the 32-bit TMEM scale word) at bits 29..30 (A) and 4..5 (B).
-    return ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
-           (sf_id << 29) | (sf_id << 4);
+    // (byte of the 32-bit TMEM scale word) at bits 29..30 (A) and 4..5 (B)
+    return ((uint32_t)(n >> 3) << 17) | (1u << 23) | (16u << 24) | (sf_id << 29) | (sf_id << 4);
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const Params p) {
+__device__ __forceinline__ float swiglu_value(float g, float u, float alpha) {
+    const float gq = __fmul_rn(g, alpha);
+    const float uq = __fmul_rn(u, alpha);
+    const float den = fminf(1.0f + __expf(-gq), 1e30f);
+    return __fmul_rn(__fdividef(gq, den), uq);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmW,
+                             const __grid_constant__ CUtensorMap tmX32,
+                             const __grid_constant__ CUtensorMap tmX64, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *empty = full + STAGES;
+    uint64_t *empty = full + SCALE_SETS * STAGES;
     uint64_t *sf_full = empty + STAGES;
     uint64_t *sf_loaded = sf_full + STAGES;
-    uint64_t *acc_full = sf_loaded + STAGES;
+    uint64_t *acc_full = sf_loaded + SCALE_SETS * STAGES;
     uint64_t *acc_empty = acc_full + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int32_t *abort_flag = reinterpret_cast<int32_t *>(smem + OFF_MISC + 4);
-    int32_t *prefix = reinterpret_cast<int32_t *>(smem + OFF_PREFIX);
+    int4 *gtab = reinterpret_cast<int4 *>(smem + OFF_GTAB);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
-    // ---- tile prefix over the groups (all threads) ----
+    // ---- per-group tile table (both CTAs compute the same one) ----
     const int G = p.G;
-    for (int g = threadIdx.x; g < G; g += NUM_THREADS) {
-        int64_t tiles;
-        if (p.group_axis == NVFP4MOE_GROUP_M) {
-            int64_t mt = ((int64_t)p.group_off[g + 1] - p.group_off[g]) / BM;
-            int64_t nt = (p.epi == EPI_SWIGLU_AMAX) ? p.f_out / 128 : p.N / BN;
-            tiles = mt * nt;
-        } else {
-            tiles = (p.M / BM) * (p.N / BN);
+    const int32_t npairs32 = (int32_t)npairs;
+    for (int g = threadIdx.x; g <= G; g += NUM_THREADS) {
+        int4 e = make_int4(0, 0, 0, 0);
+        if (g < G) {
+            const int32_t o0 = p.group_off[g], o1 = p.group_off[g + 1];
+            const bool gm = p.group_axis == NVFP4MOE_GROUP_M;
+            const int32_t rows = gm ? ((o1 - o0) / 128) * 128 : (int32_t)p.x_rows;
+            const int32_t nx = x_tiles(rows);
+            e.x = p.wtiles * nx;
+            e.y = o0;
+            e.z = nx | (x_tile_rows(rows, nx) << 16);
+            e.w = gm ? rows : (o1 - o0) / 128;
         }
-        prefix[g + 1] = (int32_t)tiles;
+        gtab[g] = e;
     }
-    if (threadIdx.x == 0) {
-        prefix[0] = 0;
-        *abort_flag = 0;
-    }
+    if (threadIdx.x == 0) *abort_flag = 0;
     __syncthreads();
-    if (warp == 0) {
-        // inclusive scan of prefix[1..G] in chunks of `per` entries per lane
-        const int per = (G + 31) / 32;
-        int32_t s = 0;
-        for (int i = 0; i < per; ++i) {
-            int idx = lane * per + i + 1;
-            if (idx <= G) s += prefix[idx];
-        }
-        int32_t incl = s;
-        for (int o = 1; o < 32; o <<= 1) {
-            int32_t n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += n;
-        }
-        int32_t run = incl - s;
-        for (int i = 0; i < per; ++i) {
-            int idx = lane * per + i + 1;
-            if (idx <= G) {
-                run += prefix[idx];
-                prefix[idx] = run;
-            }
-        }
-    }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_holder, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&sf_full[s], 4);
+            mbar_init(&sf_full[s], SF_FULL_COUNT);
+        }
+        for (int s = 0; s < SCALE_SETS * STAGES; ++s) {
+            mbar_init(&full[s], FULL_COUNT);
             mbar_init(&sf_loaded[s], 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 8);
+        mbar_init(acc_empty, ACC_EMPTY_COUNT);
         fence_mbarrier_init();
     }
+    // both CTAs' barriers exist before any arrival from the other CTA
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
-    const int64_t total = prefix[G];
     const bool nvf4 = p.kind == 0;
-    const uint32_t sfa_bytes = nvf4 ? 2048u : 512u;  // per 128-row block per stage
-    const uint32_t op_tx = A_STAGE + B_STAGE;
+    const bool swiglu = p.epi == EPI_SWIGLU_AMAX;
 
     if (warp == 0) {
         // ======================= TMA producer =======================
         if (lane == 0) {
-            prefetch_tmap(&tmA);
-            prefetch_tmap(&tmB);
+            prefetch_tmap(&tmW);
+            prefetch_tmap(&tmX32);
+            prefetch_tmap(&tmX64);
+            const uint32_t cfull = cluster_addr(full, 0);
+            const uint32_t sfc = nvf4 ? 4 : 1;  // scale chunks per k-block
             int s = 0;
-            uint32_t phase = 0;
-            for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-                const Tile T = tile_info(p, prefix, t);
-                for (int kt = 0; kt < T.kt; ++kt) {
-                    if (!wait_or_abort(&empty[s], phase ^ 1u, abort_flag, WAIT_GEMM_EMPTY)) break;
-                    // scales first, on their own barrier: they are small, land
-                    // early, and the scale warps move them into TMEM while the
-                    // operand tiles are still in flight
-                    // (NVFP4 stage = 4 chunks (256 K) per 128 rows; MXFP8 = 1 chunk (128 K))
-                    const int64_t kc = nvf4 ? (int64_t)kt * 4 : (T.k0 / 128 + kt);
-                    const uint8_t *srcA = p.a_sc + ((T.a_row / 128) * p.a_nkc + kc) * 512;
-                    const uint8_t *srcB0 = p.b_sc + ((T.b_row0 / 128) * p.b_nkc + kc) * 512;
-                    const uint8_t *srcB1 = p.b_sc + ((T.b_row1 / 128) * p.b_nkc + kc) * 512;
-                    uint8_t *ssfa = smem + OFF_SFA + s * SFA_STAGE;
-                    uint8_t *ssfb = smem + OFF_SFB + s * SFB_STAGE;
-                    mbar_arrive_expect_tx(&sf_loaded[s], 3 * sfa_bytes);
-                    bulk_load(ssfa, srcA, sfa_bytes, &sf_loaded[s]);
-                    bulk_load(ssfb, srcB0, sfa_bytes, &sf_loaded[s]);
-                    bulk_load(ssfb + sfa_bytes, srcB1, sfa_bytes, &sf_loaded[s]);
-                    mbar_arrive_expect_tx(&full[s], op_tx);
-                    const int32_t kx = (int32_t)(T.k0 + (int64_t)kt * 128);  // byte column
-                    uint8_t *sa = smem + OFF_A + s * A_STAGE;
-                    uint8_t *sb = smem + OFF_B + s * B_STAGE;
-                    tma_load_2d(sa, &tmA, kx, (int32_t)T.a_row, &full[s]);
-                    tma_load_2d(sb, &tmB, kx, (int32_t)T.b_row0, &full[s]);
-                    tma_load_2d(sb + B_STAGE / 2, &tmB, kx, (int32_t)T.b_row1, &full[s]);
+            uint32_t phase = 0, i = 0;
+            bool ok = true;
+            for (Cursor c = cursor_first(gtab, G, (int32_t)pair); c.g < G && ok && !*abort_flag;
+                 cursor_next(gtab, G, npairs32, c)) {
+                const Tile T = cursor_tile(p, c);
+                const int64_t w_row = (int64_t)T.g * p.w_rows_group + (int64_t)T.mt * 256 + 128 * rank;
+                const uint32_t kblk_tx = 2u * W_KBLK + (uint32_t)T.n * 128u;  // both CTAs
+                const int hn = T.n / 2;  // this CTA's X rows: 32, 64 or 96
+                const int32_t xr = (int32_t)(T.x_row + (int64_t)rank * hn);
+                // X scale chunk rows of the tile: a, and a + 1 if the tile
+                // reaches into it
+                const int64_t xa = T.x_row / 128;
+                const int xcr = (int)((T.x_row + T.n - 1) / 128 - xa) + 1;
+                for (int kb0 = 0; kb0 < T.kt; kb0 += 2) {
+                    const int nkb = T.kt - kb0 >= 2 ? 2 : 1;
+                    if (!wait_or_abort(&empty[s], phase ^ 1u, abort_flag, WAIT_GEMM_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sf_bytes = (uint32_t)xcr * nkb * sfc * 512u;
+                    const uint32_t sb = stage_bar(i);
+                    uint64_t *sfbar = rank == 0 ? &full[sb] : &sf_loaded[sb];
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(&full[sb], (uint32_t)nkb * kblk_tx + sf_bytes);
+                    else
+                        mbar_arrive_expect_tx(&sf_loaded[sb], sf_bytes);
+                    const int64_t kc0 = nvf4 ? (int64_t)kb0 * 4 : (T.k0 / 128 + kb0);
+                    uint8_t *ssf = smem + OFF_SFX + s * SFX_STAGE;
+                    for (int cr = 0; cr < xcr; ++cr)
+                        bulk_load(ssf + cr * (SFX_CHUNKS * 512), p.x_sc + ((xa + cr) * p.x_nkc + kc0) * 512,
+                                  nkb * sfc * 512u, sfbar);
+                    const uint32_t cbar = cfull + 8u * sb;
+                    for (int j = 0; j < nkb; ++j) {
+                        const int32_t kx = (int32_t)(T.k0 + (int64_t)(kb0 + j) * 128);  // byte column
+                        uint8_t *sw = smem + OFF_W + s * W_STAGE + j * W_KBLK;
+                        uint8_t *sx = smem + OFF_X + s * X_STAGE + j * X_KBLK;
+                        if (swiglu)
+                            tma_load_5d_pair(sw, &tmW, kx, 0, 0, 8 * T.mt + 4 * (int32_t)rank, T.g, cbar);
+                        else
+                            tma_load_2d_pair(sw, &tmW, kx, (int32_t)w_row, cbar);
+                        if (hn >= 64) tma_load_2d_pair(sx, &tmX64, kx, xr, cbar);
+                        if (hn != 64)
+                            tma_load_2d_pair(sx + (hn >= 64 ? 8192 : 0), &tmX32, kx, xr + (hn >= 64 ? 64 : 0), cbar);
+                    }
+                    ++i;
                     if (++s == STAGES) { s = 0; phase ^= 1u; }
                 }
             }
         }
-    } else if (warp >= 2 && warp <= 5) {
+    } else if (warp >= SCALE_WARP0 && warp < EPI_WARP0) {
         // ======================= scale warps =======================
         // In a 512-byte scale chunk the word (4 scales) of row r0 + 32 r1 sits
-        // at byte r0 * 16 + r1 * 4, so lane r0 reads 16 contiguous bytes per
-        // chunk: the B words of tile rows r0 + 32 j, and from the A chunk the
-        // word of row r0 + 32 q, the only A row this lane quarter computes.
+        // at byte r0 * 16 + r1 * 4, so lane r0 reads 16 contiguous bytes per X
+        // chunk (the words of X rows r0 + 32 j) and one word of each W chunk:
+        // that of the W row TMEM lane 32 q + r0 of this CTA holds.
         const int q = warp & 3;
+        const uint32_t set = (uint32_t)(warp - SCALE_WARP0) >> 2;  // stages i with i % SCALE_SETS == set
         const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
-        int s = 0;
-        uint32_t phase = 0;
-        for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-            const Tile T = tile_info(p, prefix, t);
-            for (int kt = 0; kt < T.kt; ++kt) {
-                if (!wait_or_abort(&sf_loaded[s], phase, abort_flag, WAIT_GEMM_FULL)) break;
-                const uint8_t *ssfa = smem + OFF_SFA + s * SFA_STAGE;
-                const uint8_t *ssfb = smem + OFF_SFB + s * SFB_STAGE;
-                const uint32_t slot = lane_addr + TMEM_SF + s * SF_SLOT_COLS;
+        // this lane's W row inside its 128-row scale block; SwiGLU: lanes
+        // 0..15 hold gate rows, lanes 16..31 the up rows of the same h columns
+        const int w_rib = swiglu ? 64 * (int)rank + 16 * q + (lane & 15) : 32 * q + lane;
+        const int64_t w_up = (swiglu && lane >= 16) ? p.f_out : 0;
+        const uint32_t w_word = (uint32_t)((w_rib & 31) * 16 + (w_rib >> 5) * 4);
+        const uint32_t csf_full = cluster_addr(sf_full, 0);
+        const int chunks = nvf4 ? 4 : 1;  // scale chunks per k-block
+
+        // a pipeline stage: tile at cursor c (T), k-blocks kb0 and kb0 + 1
+        struct Stage {
+            Cursor c;
+            Tile T;
+            int kb0;
+        };
+        // next stage after `st`, skipping tiles without K
+        auto next_stage = [&](Stage &st) -> bool {
+            st.kb0 += 2;
+            if (st.kb0 < st.T.kt) return true;
+            for (cursor_next(gtab, G, npairs32, st.c); st.c.g < G; cursor_next(gtab, G, npairs32, st.c)) {
+                st.T = cursor_tile(p, st.c);
+                if (st.T.kt > 0) {
+                    st.kb0 = 0;
+                    return true;
+                }
+            }
+            return false;
+        };
+        // W scale words of the stage's k-blocks: [k-block j][MMA kb]
+        auto fetch_w = [&](const Stage &st, uint32_t (&w)[2][4]) {
+            const Tile &T = st.T;
+            const int64_t wrow = swiglu ? (int64_t)T.g * p.w_rows_group + (int64_t)T.mt * 128 + w_up
+                                        : (int64_t)T.g * p.w_rows_group + (int64_t)T.mt * 256 + 128 * rank;
+            const int nkb = T.kt - st.kb0 >= 2 ? 2 : 1;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int64_t kc = nvf4 ? (int64_t)(st.kb0 + j) * 4 : (T.k0 / 128 + st.kb0 + j);
+                const uint8_t *ws = p.w_sc + ((wrow / 128) * p.w_nkc + kc) * 512 + w_word;
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb)
+                    w[j][kb] = (j < nkb && kb < chunks) ? __ldg(reinterpret_cast<const uint32_t *>(ws + kb * 512))
+                                                       : 0u;
+            }
+        };
+        // write stage i (slot s = i % STAGES) into TMEM and hand it over
+        auto put = [&](const Stage &st, uint32_t i, const uint32_t (&w)[2][4]) -> bool {
+            const Tile &T = st.T;
+            const uint32_t s = i % STAGES, sb = stage_bar(i), par = stage_par(i);
+            // the stage's bytes landed (first CTA: operands and X scales on
+            // `full`; other CTA: its X scales on `sf_loaded`); the producer
+            // only loaded them after the MMAs that last read slot s were done
+            const bool ok = rank == 0 ? wait_or_abort(&full[sb], par, abort_flag, WAIT_GEMM_FULL)
+                                      : wait_or_abort(&sf_loaded[sb], par, abort_flag, WAIT_GEMM_SF_SLOT);
+            if (!ok) return false;
+            tc_fence_after();
+            const int nkb = T.kt - st.kb0 >= 2 ? 2 : 1;
+            // tile rows start at 128 a + 64 h: column j holds word (2h + j) % 4
+            // of chunk row (2h + j) / 4
+            const bool h = (T.x_row & 64) != 0;
+            const bool need_b = (h ? 2 : 0) + T.n / 32 > 4;
+            const uint8_t *ssf = smem + OFF_SFX + s * SFX_STAGE + lane * 16;
+            for (int j = 0; j < nkb; ++j) {
+                const uint32_t slot = lane_addr + TMEM_SF + s * SF_SLOT_COLS + j * SF_KB_COLS;
                 if (nvf4) {
-                    uint32_t b[32], a[4];
+                    uint32_t b[32];
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
-                        const uint4 b0 = *reinterpret_cast<const uint4 *>(ssfb + kb * 512 + lane * 16);
-                        const uint4 b1 = *reinterpret_cast<const uint4 *>(ssfb + 2048 + kb * 512 + lane * 16);
-                        b[8 * kb + 0] = b0.x; b[8 * kb + 1] = b0.y; b[8 * kb + 2] = b0.z; b[8 * kb + 3] = b0.w;
-                        b[8 * kb + 4] = b1.x; b[8 * kb + 5] = b1.y; b[8 * kb + 6] = b1.z; b[8 * kb + 7] = b1.w;
-                        a[kb] = *reinterpret_cast<const uint32_t *>(ssfa + kb * 512 + lane * 16 + q * 4);
+                        const int c = j * 4 + kb;
+                        const uint4 A = *reinterpret_cast<const uint4 *>(ssf + c * 512);
+                        const uint4 B = need_b ? *reinterpret_cast<const uint4 *>(ssf + (SFX_CHUNKS + c) * 512)
+                                               : make_uint4(0u, 0u, 0u, 0u);
+                        b[8 * kb + 0] = h ? A.z : A.x; b[8 * kb + 1] = h ? A.w : A.y;
+                        b[8 * kb + 2] = h ? B.x : A.z; b[8 * kb + 3] = h ? B.y : A.w;
+                        b[8 * kb + 4] = h ? B.z : B.x; b[8 * kb + 5] = h ? B.w : B.y;
+                        b[8 * kb + 6] = B.z;           b[8 * kb + 7] = B.w;
                     }
                     tmem_st_32x32b_x32(slot, b);
 #pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) tmem_st_32x32b_x1(slot + 32 + 4 * kb + q, a[kb]);
+                    for (int kb = 0; kb < 4; ++kb) tmem_st_32x32b_x1(slot + 32 + 4 * kb + q, w[j][kb]);
                 } else {
-                    // one chunk per stage: the four scale bytes of a word serve
-                    // the four MMAs (byte kb selected by the MMA's scale id)
-                    const uint4 b0 = *reinterpret_cast<const uint4 *>(ssfb + lane * 16);
-                    const uint4 b1 = *reinterpret_cast<const uint4 *>(ssfb + 512 + lane * 16);
-                    const uint32_t b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    // one chunk per k-block: the four scale bytes of a word
+                    // serve its four MMAs (byte kb selected by the scale id)
+                    const uint4 A = *reinterpret_cast<const uint4 *>(ssf + j * 512);
+                    const uint4 B = need_b ? *reinterpret_cast<const uint4 *>(ssf + (SFX_CHUNKS + j) * 512)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t b[8] = {h ? A.z : A.x, h ? A.w : A.y, h ? B.x : A.z, h ? B.y : A.w,
+                                           h ? B.z : B.x, h ? B.w : B.y, B.z, B.w};
                     tmem_st_32x32b_x8(slot, b);
-                    tmem_st_32x32b_x1(slot + 32 + q,
-                                      *reinterpret_cast<const uint32_t *>(ssfa + lane * 16 + q * 4));
+                    tmem_st_32x32b_x1(slot + 32 + q, w[j][0]);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sf_full[s]);
-                if (++s == STAGES) { s = 0; phase ^= 1u; }
             }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&sf_full[s]);
+                else mbar_arrive_cluster_relaxed(csf_full + 8u * s);
+            }
+            return true;
+        };
+        // this set's stages: i = set, set + SCALE_SETS, ...; the W words of
+        // the next one are loaded before the current one is written
+        auto skip = [&](Stage &st) -> bool {
+            bool ok = true;
+            for (int k = 0; k < SCALE_SETS && ok; ++k) ok = next_stage(st);
+            return ok;
+        };
+        Stage cur;
+        cur.c.g = 0;
+        cur.c.local = (int32_t)pair - npairs32;
+        cur.c.e = gtab[0];
+        cur.T.kt = 0;
+        cur.kb0 = 0;
+        bool more = next_stage(cur);
+        uint32_t i = 0;
+        for (uint32_t k = 0; k < set && more; ++k) {
+            more = next_stage(cur);
+            ++i;
+        }
+        uint32_t wa[2][4], wb[2][4];
+        if (more) fetch_w(cur, wa);
+        // two stages per iteration so the word buffers swap roles without
+        // register copies
+        while (more && !*abort_flag) {
+            Stage nxt = cur;
+            bool more2 = skip(nxt);
+            if (more2) fetch_w(nxt, wb);
+            if (!put(cur, i, wa)) break;
+            if (!more2 || *abort_flag) break;
+            cur = nxt;
+            i += SCALE_SETS;
+            nxt = cur;
+            more = skip(nxt);
+            if (more) fetch_w(nxt, wa);
+            if (!put(cur, i, wb)) break;
+            cur = nxt;
+            i += SCALE_SETS;
         }
     } else if (warp == 1) {
-        // ======================= MMA issuer =======================
-        if (lane == 0) {
+        // ======================= MMA issuer (first CTA) =======================
+        if (rank == 0 && lane == 0) {
+            const uint32_t c_empty = cluster_addr(empty, 0), c_acc = cluster_addr(acc_full, 0);
+            const uint64_t wdesc0 = smem_desc(smem_u32(smem + OFF_W), 16, 1024, 2);
+            const uint64_t xdesc0 = smem_desc(smem_u32(smem + OFF_X), 16, 1024, 2);
             int s = 0;
             uint32_t phase = 0, acc_phase = 0;
-            const uint32_t d_tmem = tmem_base;
-            for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-                const Tile T = tile_info(p, prefix, t);
+            bool ok = true;
+            for (Cursor c = cursor_first(gtab, G, (int32_t)pair); c.g < G && ok && !*abort_flag;
+                 cursor_next(gtab, G, npairs32, c)) {
+                const Tile T = cursor_tile(p, c);
                 if (T.kt == 0) continue;
                 if (!wait_or_abort(acc_empty, acc_phase ^ 1u, abort_flag, WAIT_GEMM_ACC_EMPTY)) break;
                 tc_fence_after();
-                bool ok = true;
-                for (int kt = 0; kt < T.kt; ++kt) {
-                    if (!wait_or_abort(&full[s], phase, abort_flag, WAIT_GEMM_FULL) ||
-                        !wait_or_abort(&sf_full[s], phase, abort_flag, WAIT_GEMM_FULL)) { ok = false; break; }
+                const uint32_t idesc4 = idesc_nvf4(T.n);
+                for (int kb0 = 0; kb0 < T.kt; kb0 += 2) {
+                    const int nkb = T.kt - kb0 >= 2 ? 2 : 1;
+                    // the scale warps arrive once the stage's scales are in
+                    // TMEM and (first CTA) its operands in shared memory
+                    if (!wait_or_abort(&sf_full[s], phase, abort_flag, WAIT_GEMM_SF_FULL)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + OFF_A + s * A_STAGE);
-                    const uint32_t sb = smem_u32(smem + OFF_B + s * B_STAGE);
+                    // descriptors advance in 16-byte units: 32 bytes of K per MMA
+                    const uint64_t wd = wdesc0 + (uint64_t)((s * W_STAGE) >> 4);
+                    const uint64_t xd = xdesc0 + (uint64_t)((s * X_STAGE) >> 4);
                     const uint32_t sf = tmem_base + TMEM_SF + s * SF_SLOT_COLS;
+                    for (int j = 0; j < nkb; ++j) {
+                        const uint32_t sfj = sf + j * SF_KB_COLS;
 #pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        const uint64_t ad = smem_desc(sa + 32 * kb, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(sb + 32 * kb, 16, 1024, 2);
-                        if (nvf4) {
-                            tc_mma_nvf4(d_tmem, ad, bd, idesc_nvf4(), sf + 32 + 4 * kb, sf + 8 * kb,
-                                        (kt | kb) != 0);
-                        } else {
-                            const uint32_t sub = (uint32_t)kb << 30;  // byte kb of the scale word
-                            tc_mma_mxf8(d_tmem, ad, bd, idesc_mxf8((uint32_t)kb), (sf + 32) | sub,
-                                        sf | sub, (kt | kb) != 0);
+                        for (int kb = 0; kb < 4; ++kb) {
+                            const uint64_t woff = (uint64_t)((j * W_KBLK + 32 * kb) >> 4);
+                            const uint64_t xoff = (uint64_t)((j * X_KBLK + 32 * kb) >> 4);
+                            const uint32_t acc = (kb0 | j | kb) != 0;
+                            if (nvf4) {
+                                tc_mma_nvf4_pair(tmem_base, wd + woff, xd + xoff, idesc4, sfj + 32 + 4 * kb,
+                                                 sfj + 8 * kb, acc);
+                            } else {
+                                const uint32_t sub = (uint32_t)kb << 30;  // byte kb of the scale word
+                                tc_mma_mxf8_pair(tmem_base, wd + woff, xd + xoff, idesc_mxf8(T.n, (uint32_t)kb),
+                                                 (sfj + 32) | sub, sfj | sub, acc);
+                            }
                         }
                     }
-                    tc_commit(&empty[s]);
+                    tc_commit_pair_mc(c_empty + 8u * s, 0x3);
                     if (++s == STAGES) { s = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit(acc_full);
+                tc_commit_pair_mc(c_acc, 0x3);
                 acc_phase ^= 1u;
             }
         }
-    } else {
+    } else if (warp >= EPI_WARP0) {
         // ======================= epilogue =======================
-        const int q = warp & 3;          // TMEM lane quarter this warp may access
-        const int half = (warp - 6) >> 2;
-        const int row_in_tile = q * 32 + lane;
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int half = (warp - EPI_WARP0) >> 2;
         const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+        const uint32_t c_acc_empty = cluster_addr(acc_empty, 0);
+        const bool up_lane = lane >= 16;
+        const bool f32_out = p.epi == EPI_STORE_F32;
         uint32_t acc_phase = 0;
-        for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-            const Tile T = tile_info(p, prefix, t);
-            const int64_t row = T.out_row + row_in_tile;
+        for (Cursor c = cursor_first(gtab, G, (int32_t)pair); c.g < G && !*abort_flag;
+             cursor_next(gtab, G, npairs32, c)) {
+            const Tile T = cursor_tile(p, c);
             float alpha = 1.0f;
-            if (nvf4) alpha = __fmul_rn(p.a_ts[(int64_t)T.g * p.a_ts_stride], p.b_ts[T.g]);
+            if (nvf4) alpha = __fmul_rn(p.x_ts[(int64_t)T.g * p.x_ts_stride], p.w_ts[T.g]);
             const bool have_acc = T.kt > 0;
+            // this warp's accumulator columns (X rows): [c0, c0 + n/2), in
+            // blocks of 32
+            const int c0 = half * (T.n / 2);
+            const int nblk = T.n / 64;
+            const int64_t row0 = T.out_row + c0;  // output row of column c0
             if (have_acc) {
                 if (!wait_or_abort(acc_full, acc_phase, abort_flag, WAIT_GEMM_ACC_FULL)) break;
                 tc_fence_after();
             }
-            if (p.epi == EPI_SWIGLU_AMAX) {
-                // two rounds of (32 gate + 32 up) columns; the accumulator goes
-                // back to the MMA warp once the second round is in registers
-                uint16_t *h = static_cast<uint16_t *>(p.c);
-                float amax = 0.0f;
-                uint32_t pk[2][16];
+            float amax = 0.0f;
+            const int64_t hc = (int64_t)T.mt * 128 + 64 * rank + 16 * q + (lane & 15);  // SwiGLU
+            const int64_t col = (int64_t)T.mt * 256 + 128 * rank + 32 * q + lane;     // stores
+            // finish block b from its 32 accumulator columns v into bf16 pairs
+            // pk (SwiGLU: 8 pairs = 16 h values; store: 16 pairs); fp32 output
+            // is stored at once
+            auto finish = [&](int b, const uint32_t (&v)[32], uint32_t (&pk)[16]) {
+                if (swiglu) {
+                    // lane l < 16: gate of an h column, lane l + 16: up of the
+                    // same column; the gate lane finishes X rows 0..15 of the
+                    // block, the up lane rows 16..31
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int hc = half * 64 + c * 32;
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(lane_addr + hc, g);
-                    tmem_ld_32x32b_x32(lane_addr + 128 + hc, u);
-                    tmem_wait_ld();
-                    if (c == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(acc_empty);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
+                    for (int j = 0; j < 16; j += 2) {
                         float hv[2];
 #pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const float gq = __fmul_rn(__uint_as_float(g[i + j]), alpha);
-                            const float uq = __fmul_rn(__uint_as_float(u[i + j]), alpha);
-                            const float den = fminf(1.0f + __expf(-gq), 1e30f);
-                            hv[j] = __fmul_rn(__fdividef(gq, den), uq);
+                        for (int e = 0; e < 2; ++e) {
+                            const uint32_t send = up_lane ? v[j + e] : v[16 + j + e];
+                            const uint32_t r = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+                            const float g = __uint_as_float(up_lane ? r : v[j + e]);
+                            const float u = __uint_as_float(up_lane ? v[16 + j + e] : r);
+                            hv[e] = swiglu_value(g, u, alpha);
                         }
-                        const uint32_t b0 = f32_to_bf16_bits(hv[0]), b1 = f32_to_bf16_bits(hv[1]);
-                        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(b0 << 16)),
-                                                 fabsf(__uint_as_float(b1 << 16))));
-                        pk[c][i >> 1] = b0 | (b1 << 16);
+                        const uint32_t w = bf16x2_rn(hv[0], hv[1]);
+                        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w << 16)),
+                                                 fabsf(__uint_as_float(w & 0xFFFF0000u))));
+                        pk[j >> 1] = w;
                     }
+                } else if (!f32_out) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2)
+                        pk[j >> 1] = bf16x2_rn(__fmul_rn(__uint_as_float(v[j]), alpha),
+                                               __fmul_rn(__uint_as_float(v[j + 1]), alpha));
+                } else {
+                    float *dst = static_cast<float *>(p.c) + (row0 + 32 * b) * p.ldc + col;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dst[j * p.ldc] = __fmul_rn(__uint_as_float(v[j]), alpha);
                 }
+            };
+            // store the bf16 pairs of block b
+            auto emit = [&](int b, const uint32_t (&pk)[16]) {
+                if (swiglu) {
+                    uint16_t *dst = static_cast<uint16_t *>(p.c) + (row0 + 32 * b + (up_lane ? 16 : 0)) * p.ldc + hc;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(h + row * p.ldc + T.out_col + half * 64 + c * 32);
+                    for (int j = 0; j < 16; ++j) dst[j * p.ldc] = (uint16_t)(pk[j >> 1] >> (16 * (j & 1)));
+                } else if (!f32_out) {
+                    uint16_t *dst = static_cast<uint16_t *>(p.c) + (row0 + 32 * b) * p.ldc + col;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(pk[c][4 * v], pk[c][4 * v + 1], pk[c][4 * v + 2], pk[c][4 * v + 3]);
+                    for (int j = 0; j < 32; ++j) dst[j * p.ldc] = (uint16_t)(pk[j >> 1] >> (16 * (j & 1)));
                 }
-                amax = warp_max(amax);
-                if (lane == 0) atomic_max_nonneg(p.amax + T.g, amax);
-            } else if (p.epi == EPI_STORE_BF16) {
-                // two rounds of 64 columns, converted to bf16 as they arrive
-                uint32_t pk[4][16];
+            };
+            auto release = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(c_acc_empty);
+            };
+            // at most two TMEM round trips (blocks 0 and 1, then block 2); the
+            // accumulator goes back as soon as the last block is in registers
+            uint32_t va[32], vb[32];
+            if (have_acc) {
+                tmem_ld_32x32b_x32(lane_addr + c0, va);
+                if (nblk > 1) tmem_ld_32x32b_x32(lane_addr + c0 + 32, vb);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-                for (int rd = 0; rd < 2; ++rd) {
-                    uint32_t r0[32], r1[32];
-                    if (have_acc) {
-                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64, r0);
-                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64 + 32, r1);
-                        tmem_wait_ld();
-                        if (rd == 1) {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(acc_empty);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0u;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        pk[2 * rd][i >> 1] =
-                            f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[i]), alpha)) |
-                            (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[i + 1]), alpha)) << 16);
-                        pk[2 * rd + 1][i >> 1] =
-                            f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[i]), alpha)) |
-                            (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[i + 1]), alpha)) << 16);
-                    }
-                }
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.c) + row * p.ldc +
-                                                           T.out_col + half * 128 + c * 32);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(pk[c][4 * v], pk[c][4 * v + 1], pk[c][4 * v + 2], pk[c][4 * v + 3]);
+                for (int k = 0; k < 32; ++k) va[k] = vb[k] = 0u;
+            }
+            if (nblk <= 2) {
+                if (have_acc) release();
+                uint32_t pk[16];
+                finish(0, va, pk);
+                emit(0, pk);
+                if (nblk > 1) {
+                    finish(1, vb, pk);
+                    emit(1, pk);
                 }
             } else {
-                // fp32 out: two rounds of 64 columns stored as they arrive
-#pragma unroll
-                for (int rd = 0; rd < 2; ++rd) {
-                    uint32_t r0[32], r1[32];
-                    if (have_acc) {
-                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64, r0);
-                        tmem_ld_32x32b_x32(lane_addr + half * 128 + rd * 64 + 32, r1);
-                        tmem_wait_ld();
-                        if (rd == 1) {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(acc_empty);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0u;
-                    }
-                    float *cp = static_cast<float *>(p.c) + row * p.ldc + T.out_col + half * 128 + rd * 64;
-                    float4 *d0 = reinterpret_cast<float4 *>(cp);
-                    float4 *d1 = reinterpret_cast<float4 *>(cp + 32);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        d0[v] = make_float4(__fmul_rn(__uint_as_float(r0[4 * v]), alpha),
-                                            __fmul_rn(__uint_as_float(r0[4 * v + 1]), alpha),
-                                            __fmul_rn(__uint_as_float(r0[4 * v + 2]), alpha),
-                                            __fmul_rn(__uint_as_float(r0[4 * v + 3]), alpha));
-                        d1[v] = make_float4(__fmul_rn(__uint_as_float(r1[4 * v]), alpha),
-                                            __fmul_rn(__uint_as_float(r1[4 * v + 1]), alpha),
-                                            __fmul_rn(__uint_as_float(r1[4 * v + 2]), alpha),
-                                            __fmul_rn(__uint_as_float(r1[4 * v + 3]), alpha));
-                    }
+                uint32_t p0[16], p1[16];
+                finish(0, va, p0);
+                finish(1, vb, p1);
+                if (have_acc) {
+                    tmem_ld_32x32b_x32(lane_addr + c0 + 64, va);
+                    tmem_wait_ld();
+                    release();
                 }
+                emit(0, p0);
+                emit(1, p1);
+                finish(2, va, p0);
+                emit(2, p0);
             }
             if (have_acc) acc_phase ^= 1u;
+            if (swiglu) {
+                amax = warp_max(amax);
+                if (lane == 0) atomic_max_nonneg(p.amax + T.g, amax);
+            }
         }
     }
 
+    // No CTA leaves (or frees TMEM) while the other may still arrive on its
+    // barriers or the MMA may still write its TMEM.
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
@@ -537,28 +725,61 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// A [rows x cols_bytes] uint8 matrix, 128-byte x 128-row boxes, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols_bytes) {
+// A [rows x cols_bytes] uint8 matrix read in boxes of 128 bytes x box_rows
+// rows with 128-byte swizzle.
+bool make_map_2d(CUtensorMap *m, const void *base, int64_t rows, int64_t cols_bytes,
+                 uint32_t box_rows) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols_bytes, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols_bytes};
-    cuuint32_t box[2] = {128, 128};
+    cuuint32_t box[2] = {128, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
+// The [E x 2f x cols_bytes] gate/up weights seen as 5-D (bytes, 16 rows,
+// gate|up, 16-row group of h columns, expert), so that one box of
+// (128, 16, 2, 4, 1) brings 4 x (16 gate rows, the 16 matching up rows): 128
+// rows in the order the SwiGLU epilogue pairs them.
+bool make_map_swiglu(CUtensorMap *m, const void *base, int64_t E, int64_t f, int64_t cols_bytes) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t rb = (cuuint64_t)cols_bytes;
+    cuuint64_t dims[5] = {rb, 16, 2, (cuuint64_t)(f / 16), (cuuint64_t)E};
+    cuuint64_t strides[4] = {rb, (cuuint64_t)f * rb, 16 * rb, 2 * (cuuint64_t)f * rb};
+    cuuint32_t box[5] = {128, 16, 2, 4, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Grid: two CTAs for every cluster the device keeps resident at once (the
+// tile loop is persistent, so a cluster left waiting for a free pair of SMs
+// would double the tail).
+int pair_grid() {
     static int n = 0;
-    if (!n) {
-        int dev = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0, sms = 0;
         cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 1) sms = 148;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(sms & ~1));
+        cfg.blockDim = dim3(NUM_THREADS);
+        cfg.dynamicSmemBytes = SMEM_ALLOC;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel, &cfg) != cudaSuccess ||
+            clusters <= 0) {
+            cudaGetLastError();
+            clusters = sms / 2;
+        }
+        n = 2 * (clusters < sms / 2 ? clusters : sms / 2);
+    });
     return n;
 }
 
@@ -566,42 +787,52 @@ int sm_count() {
 
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     const bool nvf4 = a.kind == 0;
+    const bool swiglu = a.epi == EPI_SWIGLU_AMAX;
+    if (swiglu && (!nvf4 || a.group_axis != NVFP4MOE_GROUP_M || (a.N / 2) % 128 != 0))
+        return cudaErrorInvalidValue;
+    if (a.N % 256 != 0) return cudaErrorInvalidValue;
+    // the per-group tile table packs the X-tile count of a group into 16 bits
+    if (a.a_rows >= (int64_t)MAX_N * 65535) return cudaErrorInvalidValue;
     Params p{};
     p.kind = a.kind;
     p.epi = a.epi;
     p.group_axis = a.group_axis;
-    p.a_sc = a.a_sc;
-    p.b_sc = a.b_sc;
-    p.a_ts = a.a_ts;
-    p.b_ts = a.b_ts;
-    p.a_ts_stride = a.a_ts_stride;
+    // X = the token-side operand (argument "a"), W = the weights (argument "b")
+    p.x_sc = a.a_sc;
+    p.w_sc = a.b_sc;
+    p.x_ts = a.a_ts;
+    p.w_ts = a.b_ts;
+    p.x_ts_stride = a.a_ts_stride;
     p.group_off = a.group_off;
     p.G = a.G;
-    p.M = a.M;
-    p.N = a.N;
-    p.f_out = (a.epi == EPI_SWIGLU_AMAX) ? a.N / 2 : a.N;
+    p.x_rows = a.M;
+    p.f_out = swiglu ? a.N / 2 : a.N;
     p.ldc = p.f_out;
-    p.b_rows_per_group = a.b_rows_per_group;
+    p.w_rows_group = (a.group_axis == NVFP4MOE_GROUP_M) ? a.b_rows_per_group : 0;
+    p.wtiles = (int32_t)(swiglu ? p.f_out / 128 : a.N / 256);
     p.c = a.c;
     p.amax = a.amax;
     // contraction bytes per row and scale chunks per 128-row block
     const int64_t kbytes = nvf4 ? a.a_cols / 2 : a.a_cols;
-    p.a_nkc = nvf4 ? a.a_cols / 64 : a.a_cols / 128;
-    p.b_nkc = p.a_nkc;
+    p.x_nkc = nvf4 ? a.a_cols / 64 : a.a_cols / 128;
+    p.w_nkc = p.x_nkc;
     p.kt_total = (int32_t)(kbytes / 128);
-    const int64_t b_rows =
+    const int64_t w_rows =
         (a.group_axis == NVFP4MOE_GROUP_M) ? (int64_t)a.G * a.b_rows_per_group : a.N;
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, a.a, a.a_rows, kbytes) || !make_map(&mb, a.b, b_rows, kbytes))
+    CUtensorMap mw, mx32, mx64;
+    const bool okw = swiglu ? make_map_swiglu(&mw, a.b, a.G, p.f_out, kbytes)
+                            : make_map_2d(&mw, a.b, w_rows, kbytes, 128);
+    if (!okw || !make_map_2d(&mx32, a.a, a.a_rows, kbytes, 32) ||
+        !make_map_2d(&mx64, a.a, a.a_rows, kbytes, 64))
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel,
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    grouped_gemm_kernel<<<sm_count(), NUM_THREADS, SMEM_ALLOC, s>>>(ma, mb, p);
+    grouped_gemm_pair_kernel<<<pair_grid(), NUM_THREADS, SMEM_ALLOC, s>>>(mw, mx32, mx64, p);
     return cudaGetLastError();
 }
 

@@ -126,6 +126,38 @@ def test_grouped_nvfp4_gemm_ragged_groups(dev, lib, orc):
         _check_f32(got[sl], ref, mag)
 
 
+def test_grouped_nvfp4_gemm_tile_shapes(dev, lib, orc):
+    """Groups of 640, 128, 512 and 896 rows: token tiles of 192, 128 and 64
+    rows, tiles that start 64 rows into a 128-row scale block, and K = 768
+    (three 128-byte k-blocks: a full and a half pipeline stage); bf16 out."""
+    rows = [640, 128, 512, 896]
+    off = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
+    R, K, N, G = int(off[-1]), 768, 256, 4
+    A = _f32(synth.rows_np(7, synth.TAG_A, 0, R, K, 1.0))
+    a_parts, a_sc, a_ts, Ad = [], [], [], np.zeros((R, K))
+    for g in range(G):
+        c, s, t = _quant(orc, A[off[g]:off[g + 1]])
+        a_parts.append(c); a_sc.append(s); a_ts.append(t)
+        Ad[off[g]:off[g + 1]] = orc.nvfp4_to_f64(c, s, t, rows[g], K)
+    b_parts, b_sc, b_ts, Bd = [], [], [], []
+    for g in range(G):
+        W = _f32(synth.expert_weight_np(8, synth.TAG_W, g, N, K))
+        c, s, t = _quant(orc, W)
+        b_parts.append(c); b_sc.append(s); b_ts.append(t)
+        Bd.append(orc.nvfp4_to_f64(c, s, t, N, K))
+    c = torch.empty(R, N, dtype=torch.bfloat16, device=dev)
+    lib.nvfp4_grouped_gemm(dev_u8(np.concatenate(a_parts), dev),
+                           dev_u8(rowmajor_to_mma(np.concatenate(a_sc)), dev), dev_f32(a_ts, dev), 1,
+                           dev_u8(np.concatenate(b_parts), dev),
+                           dev_u8(rowmajor_to_mma(np.concatenate(b_sc)), dev), dev_f32(b_ts, dev),
+                           torch.tensor(off, device=dev), G, R, N, K, c)
+    sync()
+    got = host_bits(c)
+    for g in range(G):
+        sl = slice(off[g], off[g + 1])
+        _check_bf16(got[sl], orc.gemm_f64(Ad[sl], Bd[g]), orc.gemm_f64(np.abs(Ad[sl]), np.abs(Bd[g])))
+
+
 def _mx(orc, x, axis=0):
     c, s = orc.mxfp8_quantize(x, axis=axis, rounding=0)
     return c, s
@@ -155,11 +187,13 @@ def test_mxfp8_gemm_group_m(dev, lib, orc):
         _check_f32(got[sl], orc.gemm_f64(Ad[sl], Bd[g]), orc.gemm_f64(np.abs(Ad[sl]), np.abs(Bd[g])))
 
 
-def test_mxfp8_gemm_group_k(dev, lib, orc):
-    """Weight-gradient shape: C_g = A[:, off_g:off_g+1] . B[:, off_g:off_g+1]^T with an empty group."""
+@pytest.mark.parametrize("M", [256, 640])
+def test_mxfp8_gemm_group_k(dev, lib, orc, M):
+    """Weight-gradient shape: C_g = A[:, off_g:off_g+1] . B[:, off_g:off_g+1]^T with an empty
+    group; M = 640 output rows give token-side tiles of 192 and 64 rows."""
     seg = [256, 0, 128, 384]
     off = np.concatenate([[0], np.cumsum(seg)]).astype(np.int32)
-    M, N, Kt, G = 256, 256, int(off[-1]), 4
+    N, Kt, G = 256, int(off[-1]), 4
     A = _f32(synth.grad_rows_np(5, 0, M, Kt, synth.outlier_channels(5, Kt, 2)))
     Bm = _f32(synth.rows_np(6, synth.TAG_ACT, 0, N, Kt, 0.3))
     ac, asc = _mx(orc, A)
