@@ -441,6 +441,14 @@ NV_DEV void tma_load_5d_pair(void *dst, const CUtensorMap *map, int32_t c0, int3
         : "memory");
 }
 
+// Per-warpgroup register budget (all four warps of the warpgroup execute it).
+template <uint32_t N> NV_DEV void regs_shrink() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N> NV_DEV void regs_grow() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // --- tcgen05 (CTA pairs: every tcgen05 op of a kernel uses one cta_group) ----
 NV_DEV void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

@@ -20,13 +20,13 @@
 // and TMA keep shared memory busy, so each role does as few per stage as the
 // protocol allows.
 //
-// Roles (448 threads, 14 warps, in both CTAs of the pair):
+// Roles (640 threads, 20 warps, in both CTAs of the pair):
 //   warp 0       TMA producer: this CTA's W and X halves (128-byte swizzle),
 //                completion counted on the first CTA's `full` barrier, and
 //                the X block scales of the stage (plain bulk copies of the one
 //                or two 128-row chunk rows) into this CTA: counted on `full`
 //                in the first CTA, on its own `sf_loaded` in the other.
-//   warps 2..5   scale warps, one per TMEM lane quarter (SCALE_SETS sets of
+//   warps 4..7   scale warps, one per TMEM lane quarter (SCALE_SETS sets of
 //                four can take turns by stage). Each lane reads the stage's X
 //                scale words from shared memory and the W scale words of its
 //                own TMEM lane, loaded from L2 one stage ahead, and writes them
@@ -46,13 +46,12 @@
 //                wait on sf_full; one commit multicast to both CTAs' `empty`
 //                barriers per stage and, after a tile's last stage, to both
 //                `acc_full` barriers.
-//   warps 6..13  epilogue: two warps per lane quarter, n/2 accumulator
-//                columns each, read with tcgen05.ld in two round trips of at
-//                most 64 columns and packed to bf16 pairs (SwiGLU: finished to
-//                h first), so that the whole share fits in registers; the
-//                accumulator goes back to the MMA warp (arrival on the first
-//                CTA's acc_empty) as soon as the last columns are in
-//                registers, and the stores follow. Lane =
+//   warps 8..19  epilogue: three warps per lane quarter, at most two
+//                32-column blocks each, read with tcgen05.ld in one round
+//                trip; the accumulator goes back to the MMA warp (arrival on
+//                the first CTA's acc_empty) as soon as they are in registers,
+//                before any arithmetic, and SwiGLU or the bf16 / fp32
+//                conversion and the stores follow. Lane =
 //                output column, register = output row, so every store
 //                instruction of a warp writes one contiguous run of an output
 //                row.
@@ -94,9 +93,18 @@ constexpr int X_STAGE = 2 * X_KBLK;
 constexpr int SFX_CHUNKS = 8, SFX_STAGE = 2 * SFX_CHUNKS * 512;
 // scale warps come in SCALE_SETS sets of four taking turns by stage; the
 // epilogue's two warps per lane quarter follow them
+// Warpgroups: 0 = producer, MMA issuer and two idle warps; 1 = scale warps
+// (SCALE_SETS sets of four); then the epilogue, three warps per TMEM lane
+// quarter, each owning at most two 32-column blocks of a tile of up to
+// MAX_N = 192 columns. setmaxnreg moves registers from warpgroup 0 to the
+// epilogue: 128 x 48 + 128 x 96 + 384 x 120 = 64512 <= 640 x 102.
 constexpr int SCALE_SETS = 1;
-constexpr int SCALE_WARP0 = 2, EPI_WARP0 = SCALE_WARP0 + 4 * SCALE_SETS;
-constexpr int NUM_THREADS = 32 * (EPI_WARP0 + 8);
+constexpr int SCALE_WARP0 = 4, EPI_WARP0 = SCALE_WARP0 + 4 * SCALE_SETS;
+constexpr int EPI_PER_QUARTER = 3, EPI_WARPS = 4 * EPI_PER_QUARTER;
+constexpr int NUM_THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+constexpr uint32_t REGS_CONTROL = 48, REGS_EPILOGUE = 120;
+static_assert(NUM_THREADS == 640, "register split below assumes 20 warps");
+static_assert(128 * REGS_CONTROL + 128 * 96 + 32 * EPI_WARPS * REGS_EPILOGUE <= 65536, "register split");
 constexpr int MAX_GROUPS = 1024;
 constexpr uint32_t TMEM_COLS = 512, TMEM_SF = MAX_N, SF_KB_COLS = 48, SF_SLOT_COLS = 96;
 
@@ -120,7 +128,7 @@ static_assert(TMEM_SF + STAGES * SF_SLOT_COLS <= TMEM_COLS, "TMEM columns");
 
 constexpr uint32_t FULL_COUNT = 1;        // the first CTA's producer
 constexpr uint32_t SF_FULL_COUNT = 8;     // 4 scale warps x 2 CTAs
-constexpr uint32_t ACC_EMPTY_COUNT = 16;  // 8 epilogue warps x 2 CTAs
+constexpr uint32_t ACC_EMPTY_COUNT = 2 * EPI_WARPS;  // every epilogue warp of both CTAs
 
 __host__ __device__ constexpr uint32_t stage_bar(uint32_t i) {
     return (i % SCALE_SETS) * STAGES + (i / SCALE_SETS) % STAGES;
@@ -317,6 +325,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const bool swiglu = p.epi == EPI_SWIGLU_AMAX;
 
     if (warp == 0) {
+        regs_shrink<REGS_CONTROL>();
         // ======================= TMA producer =======================
         if (lane == 0) {
             prefetch_tmap(&tmW);
@@ -521,6 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             i += SCALE_SETS;
         }
     } else if (warp == 1) {
+        regs_shrink<REGS_CONTROL>();
         // ======================= MMA issuer (first CTA) =======================
         if (rank == 0 && lane == 0) {
             const uint32_t c_empty = cluster_addr(empty, 0), c_acc = cluster_addr(acc_full, 0);
@@ -575,9 +585,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
         }
     } else if (warp >= EPI_WARP0) {
+        regs_grow<REGS_EPILOGUE>();
         // ======================= epilogue =======================
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int half = (warp - EPI_WARP0) >> 2;
+        const int q = warp & 3;                   // TMEM lane quarter this warp may access
+        const int sub = (warp - EPI_WARP0) >> 2;  // which pair of 32-column blocks
         const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
         const uint32_t c_acc_empty = cluster_addr(acc_empty, 0);
         const bool up_lane = lane >= 16;
@@ -589,110 +600,93 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             float alpha = 1.0f;
             if (nvf4) alpha = __fmul_rn(p.x_ts[(int64_t)T.g * p.x_ts_stride], p.w_ts[T.g]);
             const bool have_acc = T.kt > 0;
-            // this warp's accumulator columns (X rows): [c0, c0 + n/2), in
-            // blocks of 32
-            const int c0 = half * (T.n / 2);
-            const int nblk = T.n / 64;
-            const int64_t row0 = T.out_row + c0;  // output row of column c0
+            // this warp's accumulator columns (X rows): blocks 2 sub and
+            // 2 sub + 1 of the tile's n / 32
+            const int b0 = 2 * sub;
+            const int nb = max(0, min(2, T.n / 32 - b0));
+            const int64_t row0 = T.out_row + 32 * b0;  // output row of the first column
             if (have_acc) {
                 if (!wait_or_abort(acc_full, acc_phase, abort_flag, WAIT_GEMM_ACC_FULL)) break;
                 tc_fence_after();
             }
+            uint32_t va[32], vb[32];
+            if (have_acc && nb > 0) {
+                tmem_ld_32x32b_x32(lane_addr + 32 * b0, va);
+                if (nb > 1) tmem_ld_32x32b_x32(lane_addr + 32 * b0 + 32, vb);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) va[k] = vb[k] = 0u;
+            }
+            if (have_acc) {
+                // the accumulator goes back before any arithmetic
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(c_acc_empty);
+                acc_phase ^= 1u;
+            }
             float amax = 0.0f;
-            const int64_t hc = (int64_t)T.mt * 128 + 64 * rank + 16 * q + (lane & 15);  // SwiGLU
-            const int64_t col = (int64_t)T.mt * 256 + 128 * rank + 32 * q + lane;     // stores
-            // finish block b from its 32 accumulator columns v into bf16 pairs
-            // pk (SwiGLU: 8 pairs = 16 h values; store: 16 pairs); fp32 output
-            // is stored at once
-            auto finish = [&](int b, const uint32_t (&v)[32], uint32_t (&pk)[16]) {
+            // finish and store block b (0 or 1 of this warp) from its 32
+            // accumulator columns v
+            auto finish = [&](int b, const uint32_t (&v)[32]) {
+                const int64_t r = row0 + 32 * b;  // output row of column 0 of the block
                 if (swiglu) {
                     // lane l < 16: gate of an h column, lane l + 16: up of the
                     // same column; the gate lane finishes X rows 0..15 of the
                     // block, the up lane rows 16..31
+                    const int64_t hc = (int64_t)T.mt * 128 + 64 * rank + 16 * q + (lane & 15);
+                    uint16_t *dst = static_cast<uint16_t *>(p.c) + (r + (up_lane ? 16 : 0)) * p.ldc + hc;
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) {
                         float hv[2];
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
                             const uint32_t send = up_lane ? v[j + e] : v[16 + j + e];
-                            const uint32_t r = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
-                            const float g = __uint_as_float(up_lane ? r : v[j + e]);
-                            const float u = __uint_as_float(up_lane ? v[16 + j + e] : r);
+                            const uint32_t x = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+                            const float g = __uint_as_float(up_lane ? x : v[j + e]);
+                            const float u = __uint_as_float(up_lane ? v[16 + j + e] : x);
                             hv[e] = swiglu_value(g, u, alpha);
                         }
                         const uint32_t w = bf16x2_rn(hv[0], hv[1]);
                         amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w << 16)),
                                                  fabsf(__uint_as_float(w & 0xFFFF0000u))));
-                        pk[j >> 1] = w;
+                        *dst = (uint16_t)w;
+                        dst += p.ldc;
+                        *dst = (uint16_t)(w >> 16);
+                        dst += p.ldc;
                     }
-                } else if (!f32_out) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2)
-                        pk[j >> 1] = bf16x2_rn(__fmul_rn(__uint_as_float(v[j]), alpha),
-                                               __fmul_rn(__uint_as_float(v[j + 1]), alpha));
                 } else {
-                    float *dst = static_cast<float *>(p.c) + (row0 + 32 * b) * p.ldc + col;
+                    const int64_t col = (int64_t)T.mt * 256 + 128 * rank + 32 * q + lane;
+                    if (!f32_out) {
+                        uint16_t *dst = static_cast<uint16_t *>(p.c) + r * p.ldc + col;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) dst[j * p.ldc] = __fmul_rn(__uint_as_float(v[j]), alpha);
+                        for (int j = 0; j < 32; j += 2) {
+                            const uint32_t w = bf16x2_rn(__fmul_rn(__uint_as_float(v[j]), alpha),
+                                                         __fmul_rn(__uint_as_float(v[j + 1]), alpha));
+                            *dst = (uint16_t)w;
+                            dst += p.ldc;
+                            *dst = (uint16_t)(w >> 16);
+                            dst += p.ldc;
+                        }
+                    } else {
+                        float *dst = static_cast<float *>(p.c) + r * p.ldc + col;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            *dst = __fmul_rn(__uint_as_float(v[j]), alpha);
+                            dst += p.ldc;
+                        }
+                    }
                 }
             };
-            // store the bf16 pairs of block b
-            auto emit = [&](int b, const uint32_t (&pk)[16]) {
-                if (swiglu) {
-                    uint16_t *dst = static_cast<uint16_t *>(p.c) + (row0 + 32 * b + (up_lane ? 16 : 0)) * p.ldc + hc;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) dst[j * p.ldc] = (uint16_t)(pk[j >> 1] >> (16 * (j & 1)));
-                } else if (!f32_out) {
-                    uint16_t *dst = static_cast<uint16_t *>(p.c) + (row0 + 32 * b) * p.ldc + col;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) dst[j * p.ldc] = (uint16_t)(pk[j >> 1] >> (16 * (j & 1)));
-                }
-            };
-            auto release = [&]() {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster_relaxed(c_acc_empty);
-            };
-            // at most two TMEM round trips (blocks 0 and 1, then block 2); the
-            // accumulator goes back as soon as the last block is in registers
-            uint32_t va[32], vb[32];
-            if (have_acc) {
-                tmem_ld_32x32b_x32(lane_addr + c0, va);
-                if (nblk > 1) tmem_ld_32x32b_x32(lane_addr + c0 + 32, vb);
-                tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int k = 0; k < 32; ++k) va[k] = vb[k] = 0u;
-            }
-            if (nblk <= 2) {
-                if (have_acc) release();
-                uint32_t pk[16];
-                finish(0, va, pk);
-                emit(0, pk);
-                if (nblk > 1) {
-                    finish(1, vb, pk);
-                    emit(1, pk);
-                }
-            } else {
-                uint32_t p0[16], p1[16];
-                finish(0, va, p0);
-                finish(1, vb, p1);
-                if (have_acc) {
-                    tmem_ld_32x32b_x32(lane_addr + c0 + 64, va);
-                    tmem_wait_ld();
-                    release();
-                }
-                emit(0, p0);
-                emit(1, p1);
-                finish(2, va, p0);
-                emit(2, p0);
-            }
-            if (have_acc) acc_phase ^= 1u;
+            if (nb > 0) finish(0, va);
+            if (nb > 1) finish(1, vb);
             if (swiglu) {
                 amax = warp_max(amax);
-                if (lane == 0) atomic_max_nonneg(p.amax + T.g, amax);
+                if (lane == 0 && nb > 0) atomic_max_nonneg(p.amax + T.g, amax);
             }
         }
+    } else {
+        regs_shrink<REGS_CONTROL>();  // warps 2 and 3: idle
     }
 
     // No CTA leaves (or frees TMEM) while the other may still arrive on its
