@@ -36,10 +36,11 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 expert-FFN fwd TFLOPS (% of B200 FP4 peak); quantizer HBM GB/s"
-# dram__bytes_read.sum + dram__bytes_write.sum of moe_expert_fwd's kernels per
-# call, from the ncu capture summarised in profiles/; None until captured for
-# the current kernels.
-EXPERT_FWD_DRAM_BYTES = None
+# dram__bytes_read.sum + dram__bytes_write.sum of moe_expert_fwd's three
+# kernels (GEMM1 + SwiGLU 5.745 GB, requantize 0.952 GB, GEMM2 3.66 GB) per
+# call of the full-size layer, from a 1-pass ncu capture of the CTA-pair GEMM
+# (summary under profiles/). Set back to None when those kernels change.
+EXPERT_FWD_DRAM_BYTES = 10.357e9
 
 
 def load_peaks():
@@ -488,7 +489,9 @@ def main():
     achieved = flops / (ex_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak, 1),
                 "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
-                "traffic": EXPERT_FWD_DRAM_BYTES,
+                "traffic": EXPERT_FWD_DRAM_BYTES if args.workload == "full_moe" else None,
+                "traffic_frac_hbm": (round(EXPERT_FWD_DRAM_BYTES / (ex_ms * 1e-3) / (peaks["hbm_gbs"] * 1e9), 4)
+                                     if args.workload == "full_moe" else None),
                 "kernel": "moe_expert_fwd (grouped GEMM1+SwiGLU+amax, requantize, grouped GEMM2)",
                 "peak_source": f"{peaks['source']} bf16 sustained x 4 (nominal FP4:BF16 ratio)",
                 "weights_hbm_floor_ms": round(0.5625 * 3 * d * f * E / (peaks["hbm_gbs"] * 1e6), 3)}

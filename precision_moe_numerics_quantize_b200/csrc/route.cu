@@ -20,9 +20,11 @@ namespace nvfp4moe {
 static constexpr int CHUNK = 1024;
 
 // ---------------------------------------------------------------------------
-// 1. top-k: each lane owns experts lane, lane + 32, ...; k rounds of a warp
-// argmax (largest logit, ties to the lower expert id).
+// 1. top-k: one warp per token; lane l owns experts l, l + 32, ... (PER of
+// them); k rounds of a warp argmax (largest logit, ties to the lower expert
+// id). Lane j keeps the j-th choice, so nothing is indexed at run time.
 // ---------------------------------------------------------------------------
+template <int PER>
 __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int64_t T,
                                                    int32_t E, int32_t k, int renorm,
                                                    int32_t *__restrict__ idx_out,
@@ -31,25 +33,23 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
     const int64_t t = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
     const float *l = logits + t * E;
-    constexpr int MAXPER = 32;  // E <= 1024
-    float v[MAXPER];
-    const int per = (E + 31) / 32;
+    const float ninf = __int_as_float(0xff800000);
+    float v[PER];
 #pragma unroll
-    for (int i = 0; i < MAXPER; ++i) {
-        int e = lane + 32 * i;
-        v[i] = (i < per && e < E) ? l[e] : __int_as_float(0xff800000);
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? __ldg(l + e) : ninf;
     }
     uint32_t taken = 0;  // bit i: element i of this lane already chosen
-    float sel_l[32];
-    int sel_e[32];
-    float mx = 0.0f;
+    float my_l = 0.0f, mx = 0.0f;
+    int my_e = 0;
     for (int j = 0; j < k; ++j) {
-        float bv = __int_as_float(0xff800000);
+        float bv = ninf;
         int be = 0x7FFFFFFF;
 #pragma unroll
-        for (int i = 0; i < MAXPER; ++i) {
-            int e = lane + 32 * i;
-            bool ok = i < per && e < E && !((taken >> i) & 1u);
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            const bool ok = e < E && !((taken >> i) & 1u);
             if (ok && (v[i] > bv || (v[i] == bv && e < be) || be == 0x7FFFFFFF)) {
                 bv = v[i];
                 be = e;
@@ -57,42 +57,37 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
-            int oe = __shfl_xor_sync(0xFFFFFFFFu, be, o);
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+            const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, o);
             if (ov > bv || (ov == bv && oe < be)) {
                 bv = ov;
                 be = oe;
             }
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        sel_l[j] = bv;
-        sel_e[j] = be;
+        if (lane == j) {
+            my_l = bv;
+            my_e = be;
+        }
         if (j == 0) mx = bv;
     }
-    // weights: softmax over the chosen logits (renorm) or over all E
-    float denom = 0.0f;
+    // weights: softmax over the chosen logits (renorm) or over all E, each
+    // sum a fixed-order tree over the lanes
+    float s = 0.0f;
     if (renorm) {
-        for (int j = 0; j < k; ++j) denom += expf(sel_l[j] - mx);
+        s = lane < k ? expf(my_l - mx) : 0.0f;
     } else {
-        float s = 0.0f;
 #pragma unroll
-        for (int i = 0; i < MAXPER; ++i) {
-            int e = lane + 32 * i;
-            if (i < per && e < E) s += expf(v[i] - mx);
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) s += expf(v[i] - mx);
         }
-        // fixed-order tree over the lanes
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-        denom = s;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
     if (lane < k) {
-        // lane j writes slot j
-        float lj = 0.0f;
-        int ej = 0;
-        for (int j = 0; j < k; ++j)
-            if (j == lane) { lj = sel_l[j]; ej = sel_e[j]; }
-        idx_out[t * k + lane] = ej;
-        w_out[t * k + lane] = expf(lj - mx) / denom;
+        idx_out[t * k + lane] = my_e;
+        w_out[t * k + lane] = expf(my_l - mx) / s;
     }
 }
 
@@ -143,9 +138,21 @@ __global__ void __launch_bounds__(1024) offsets_kernel(int32_t *__restrict__ cou
     const int e = threadIdx.x;
     int32_t total = 0;
     if (e < E) {
-        for (int64_t c = 0; c < n_chunks; ++c) {
-            int32_t v = counts[c * E + e];
-            counts[c * E + e] = total;  // exclusive base within the expert
+        // eight independent loads in flight per round
+        int64_t c = 0;
+        for (; c + 8 <= n_chunks; c += 8) {
+            int32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = counts[(c + u) * E + e];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                counts[(c + u) * E + e] = total;  // exclusive base within the expert
+                total += v[u];
+            }
+        }
+        for (; c < n_chunks; ++c) {
+            const int32_t v = counts[c * E + e];
+            counts[c * E + e] = total;
             total += v;
         }
         expert_cnt[e] = total;
@@ -240,15 +247,16 @@ __global__ void __launch_bounds__(256) dispatch_quant_kernel(
     }
 }
 
+// One CTA per expert: its padding rows are [off_e + cnt_e, off_{e+1}).
 __global__ void __launch_bounds__(256) zero_pad_rows_kernel(
-    const int32_t *__restrict__ token_of, const int32_t *__restrict__ expert_off, int32_t E,
-    int64_t d, uint8_t *__restrict__ xq, uint8_t *__restrict__ xq_sc) {
-    const int64_t rows = expert_off[E];
+    const int32_t *__restrict__ expert_cnt, const int32_t *__restrict__ expert_off, int64_t d,
+    uint8_t *__restrict__ xq, uint8_t *__restrict__ xq_sc) {
+    const int e = blockIdx.x;
+    const int64_t r0 = (int64_t)expert_off[e] + expert_cnt[e];
+    const int64_t n = (int64_t)expert_off[e + 1] - r0;
     const int64_t G = d / 64;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / G, g = i - r * G;
-        if (token_of[r] >= 0) continue;
+    for (int64_t i = threadIdx.x; i < n * G; i += blockDim.x) {
+        const int64_t r = r0 + i / G, g = i % G;
         uint4 *co = reinterpret_cast<uint4 *>(xq + r * (d / 2) + g * 32);
         co[0] = make_uint4(0, 0, 0, 0);
         co[1] = make_uint4(0, 0, 0, 0);
@@ -331,8 +339,18 @@ cudaError_t launch_route_permute(const float *logits, const uint16_t *x, int64_t
     if ((e = cudaMemsetAsync(token_of, 0xFF, sizeof(int32_t) * rows_alloc, s)) != cudaSuccess)
         return e;
     if (T > 0) {
-        topk_kernel<<<(unsigned)((T + 7) / 8), 256, 0, s>>>(logits, T, E, k, renorm, topk_idx,
-                                                          topk_w);
+        const unsigned tgrid = (unsigned)((T + 7) / 8);
+        const int per = (E + 31) / 32;
+        if (per <= 4)
+            topk_kernel<4><<<tgrid, 256, 0, s>>>(logits, T, E, k, renorm, topk_idx, topk_w);
+        else if (per <= 8)
+            topk_kernel<8><<<tgrid, 256, 0, s>>>(logits, T, E, k, renorm, topk_idx, topk_w);
+        else if (per <= 12)
+            topk_kernel<12><<<tgrid, 256, 0, s>>>(logits, T, E, k, renorm, topk_idx, topk_w);
+        else if (per <= 16)
+            topk_kernel<16><<<tgrid, 256, 0, s>>>(logits, T, E, k, renorm, topk_idx, topk_w);
+        else
+            topk_kernel<32><<<tgrid, 256, 0, s>>>(logits, T, E, k, renorm, topk_idx, topk_w);
         const int warps = 4;
         chunk_rank_kernel<<<(unsigned)((nc + warps - 1) / warps), 32 * warps,
                             warps * E * sizeof(int32_t), s>>>(topk_idx, n_slots, E, counts,
@@ -352,8 +370,7 @@ cudaError_t launch_route_permute(const float *logits, const uint16_t *x, int64_t
                                                                     xq_sc, x_ts, 1);
     else
         dispatch_quant_kernel<<<1, 32, 0, s>>>(x, 0, d, k, amax_use, pos, xq, xq_sc, x_ts, 1);
-    zero_pad_rows_kernel<<<grid_cap(rows_alloc * (d / 64)), 256, 0, s>>>(token_of, expert_off, E,
-                                                                        d, xq, xq_sc);
+    zero_pad_rows_kernel<<<E, 256, 0, s>>>(expert_cnt, expert_off, d, xq, xq_sc);
     return cudaGetLastError();
 }
 
