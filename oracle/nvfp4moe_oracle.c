@@ -502,6 +502,55 @@ ORACLE_API void oracle_rht32_dequantize(const uint8_t *codes, const uint8_t *sca
     free(v);
 }
 
+/*
+ * Combine straight from the RHT32-quantized payload (aicoder.com 'Key
+ * Takeaways': the combine traffic travels block-scaled after a 32-point random
+ * Hadamard transform).
+ * READING: the transform is linear, so the weighted sum of a token's k rows is
+ * taken in the transformed domain and one inverse transform per token
+ * follows: sum_j w_j H^-1 v_j = H^-1 sum_j w_j v_j. Values are the exact
+ * dequantized payload (NVFP4: e2m1 * e4m3 scale * ts; MXFP8: e4m3 * 2^k),
+ * summed and transformed in fp64 (c = 1/sqrt(32) in fp64), rounded once to
+ * bf16 (oracle_combine_rht) or returned in fp64 (oracle_combine_rht_f64).
+ * codes/scales: rows x d payload in the ROWMAJOR layout of oracle_rht32_quantize.
+ */
+static double payload_value(const uint8_t *codes, const uint8_t *scales, float ts, int fmt,
+                            int64_t d, int64_t r, int64_t c) {
+    if (fmt == 0) {
+        uint8_t byte = codes[r * (d / 2) + c / 2];
+        uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 15);
+        return oracle_e2m1_decode(nib) * oracle_e4m3_decode(scales[r * (d / 16) + c / 16]) * (double)ts;
+    }
+    return oracle_e4m3_decode(codes[r * d + c]) * oracle_e8m0_decode(scales[r * (d / 32) + c / 32]);
+}
+
+ORACLE_API void oracle_combine_rht_f64(const uint8_t *codes, const uint8_t *scales, float ts,
+                                       int fmt, uint64_t sign_seed, const int32_t *pos,
+                                       const double *w, int64_t T, int32_t k, int64_t d,
+                                       double *out) {
+    uint32_t s = oracle_rht_signs(sign_seed);
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t b = 0; b < d / 32; ++b) {
+            double acc[32];
+            for (int i = 0; i < 32; ++i) {
+                double sum = 0.0;
+                for (int j = 0; j < k; ++j)
+                    sum += w[t * k + j] * payload_value(codes, scales, ts, fmt, d, pos[t * k + j], b * 32 + i);
+                acc[i] = sum;
+            }
+            oracle_rht32_f64(acc, s, 1, out + t * d + b * 32);
+        }
+}
+
+ORACLE_API void oracle_combine_rht(const uint8_t *codes, const uint8_t *scales, float ts, int fmt,
+                                   uint64_t sign_seed, const int32_t *pos, const double *w,
+                                   int64_t T, int32_t k, int64_t d, uint16_t *out_bits) {
+    double *x = (double *)malloc(sizeof(double) * (size_t)(T * d));
+    oracle_combine_rht_f64(codes, scales, ts, fmt, sign_seed, pos, w, T, k, d, x);
+    for (int64_t i = 0; i < T * d; ++i) out_bits[i] = oracle_bf16_from_f64(x[i]);
+    free(x);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Routing and permutation ([P4] "PART 01": 384 experts, 8 routed per token) */
 /* ------------------------------------------------------------------------ */

@@ -16,7 +16,7 @@ __all__ = [
     "nvfp4_to_f64", "philox4x32_10", "philox_word", "mxfp8_quantize", "mxfp8_dequantize",
     "rht_signs", "rht32_forward_f32", "rht32_inverse_f32", "rht32_f64", "rht32_quantize",
     "rht32_dequantize", "route", "permute", "gemm_f64", "swiglu", "expert_ffn", "combine",
-    "combine_f32", "mxfp8_rpad",
+    "combine_f32", "combine_rht", "mxfp8_rpad",
 ]
 
 _lib = None
@@ -68,6 +68,10 @@ def _declare(L):
                                      _P, C.c_float, _P, _I64, _P, _P, _P, _P, _P]),
         "oracle_combine": (None, [_P, _P, _P, _I64, _I32, _I64, _P]),
         "oracle_combine_f32": (None, [_P, _P, _P, _I64, _I32, _I64, _P]),
+        "oracle_combine_rht": (None, [_P, _P, C.c_float, C.c_int, _U64, _P, _P, _I64, _I32,
+                                      _I64, _P]),
+        "oracle_combine_rht_f64": (None, [_P, _P, C.c_float, C.c_int, _U64, _P, _P, _I64,
+                                          _I32, _I64, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -251,6 +255,26 @@ def rht32_dequantize(codes, scales, ts, rows, cols, sign_seed, fmt):
     out = np.zeros((rows, cols), np.float32)
     lib().oracle_rht32_dequantize(_p(codes), _p(scales), float(ts or 0.0), rows, cols, sign_seed,
                                   fmt, _p(out))
+    return out
+
+
+def combine_rht(codes, scales, ts, fmt, sign_seed, pos, w, f64=False):
+    """Combine straight from an RHT32-quantized payload (rows x d, ROWMAJOR
+    scales): bf16 bits [T, d], or the fp64 values before rounding."""
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    pos = _c(pos, np.int32)
+    w = _c(w, np.float64)
+    T, k = pos.shape
+    d = scales.shape[1] * (16 if fmt == 0 else 32)
+    if f64:
+        out = np.zeros((T, d), np.float64)
+        lib().oracle_combine_rht_f64(_p(codes), _p(scales), float(ts or 0.0), fmt, sign_seed,
+                                     _p(pos), _p(w), T, k, d, _p(out))
+    else:
+        out = np.zeros((T, d), np.uint16)
+        lib().oracle_combine_rht(_p(codes), _p(scales), float(ts or 0.0), fmt, sign_seed,
+                                 _p(pos), _p(w), T, k, d, _p(out))
     return out
 
 

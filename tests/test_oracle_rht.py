@@ -97,3 +97,81 @@ def test_nvfp4_payload_amax_is_over_transformed_values(orc):
     assert ts == np.float32(np.float32(np.abs(v).max()) / np.float32(2688.0))
     c2, sc2, ts2 = orc.nvfp4_quantize(v)
     assert np.array_equal(c, c2) and np.array_equal(sc, sc2)
+
+
+# -- combine straight from the quantized payload --------------------------------
+
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]  # the E2M1 grid, from the format
+
+
+def _decode_payload(codes, scales, ts, fmt, d):
+    """Dequantized payload rows in fp64, written out from the format
+    definitions (E2M1 grid above, E4M3 through torch's float8_e4m3fn, E8M0 as
+    a power of two), independent of the oracle's decoders."""
+    import torch
+    rows = codes.shape[0]
+    if fmt == 0:
+        lo, hi = codes & 15, codes >> 4
+        nib = np.stack([lo, hi], axis=2).reshape(rows, d)
+        mag = np.array(E2M1_VALUES)[nib & 7]
+        val = np.where(nib & 8, -mag, mag)
+        sf = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        return val * np.repeat(sf, 16, axis=1) * float(ts)
+    e4 = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return e4 * np.repeat(np.exp2(scales.astype(np.float64) - 127.0), 32, axis=1)
+
+
+def _combine_case(orc, fmt, T=6, k=3, d=128, seed=3):
+    R = T * k
+    x = synth.bf16_bits_to_f32(synth.payload_rows_np(seed, 0, R, d, synth.outlier_channels(seed, d, 2)))
+    codes, scales, ts = orc.rht32_quantize(x, 11, fmt)
+    rng = np.random.default_rng(seed)
+    pos = rng.permutation(R).astype(np.int32).reshape(T, k)
+    w = rng.random((T, k))
+    w /= w.sum(axis=1, keepdims=True)
+    return codes, scales, ts, pos, w
+
+
+def test_combine_rht_equals_explicit_hadamard_arithmetic(orc):
+    """oracle_combine_rht = s * (H32 @ sum_j w_j v_j) / sqrt(32) per 32-block,
+    with H32 from scipy and the payload decoded from the format definitions."""
+    import torch
+    H = scipy.linalg.hadamard(32).astype(np.float64)
+    s = orc.rht_signs(11)
+    sv = np.array([-1.0 if (s >> i) & 1 else 1.0 for i in range(32)])
+    for fmt in (0, 1):
+        d = 128
+        codes, scales, ts, pos, w = _combine_case(orc, fmt, d=d)
+        v = _decode_payload(codes, scales, ts, fmt, d)
+        T, k = pos.shape
+        ref = np.zeros((T, d))
+        for t in range(T):
+            acc = sum(w[t, j] * v[pos[t, j]] for j in range(k))
+            for b in range(d // 32):
+                ref[t, b * 32:(b + 1) * 32] = sv * (H @ acc[b * 32:(b + 1) * 32]) / np.sqrt(32.0)
+        got = orc.combine_rht(codes, scales, ts, fmt, 11, pos, w, f64=True)
+        scale = np.abs(ref).max()
+        assert np.abs(got - ref).max() <= 1e-12 * scale
+        bits = orc.combine_rht(codes, scales, ts, fmt, 11, pos, w)
+        tb = torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+        # bit-equal away from exact cancellation (there fp64 rounding order
+        # decides the sign of a ~1e-15 value)
+        big = np.abs(ref) > 1e-9 * scale
+        assert np.array_equal(bits[big], tb[big])
+
+
+def test_combine_rht_is_the_combine_of_the_inverted_rows(orc):
+    """Linearity: transforming once after the weighted sum equals combining the
+    per-row inverse transforms (oracle_rht32_dequantize in fp32, then
+    oracle_combine_f32) up to the fp32 rounding of those rows."""
+    for fmt in (0, 1):
+        d = 128
+        codes, scales, ts, pos, w = _combine_case(orc, fmt, d=d, seed=5)
+        R = pos.size
+        rows = orc.rht32_dequantize(codes, scales, ts, R, d, 11, fmt)
+        via_rows = synth.bf16_bits_to_f32(orc.combine_f32(rows, pos, w)).astype(np.float64)
+        once = synth.bf16_bits_to_f32(orc.combine_rht(codes, scales, ts, fmt, 11, pos, w)).astype(np.float64)
+        mag = np.abs(once).max()
+        assert np.abs(via_rows - once).max() <= 2 ** -8 * mag
+        # and the two agree to the last bit on most elements
+        assert np.mean(via_rows == once) > 0.9
