@@ -228,6 +228,31 @@ def companions(M, synth, torch, dev, L, peaks, reps=10):
         res[name] = {"ms": round(ms, 4), "GB/s": round(g, 1), "frac_hbm": round(g / hbm, 3),
                      "elements": elems, "algorithmic_bytes_per_elem": bytes_per_elem}
 
+    # The same layer under the Zipf-skewed router (Gumbel-top-k over a Zipf(1.1)
+    # expert popularity): a few experts take thousands of rows, many only tens.
+    zl = torch.from_numpy(synth.logits_zipf_np(2, T, E)).to(dev)
+    saved = L["logits"]
+    L["logits"] = zl
+    zcalls = layer_calls(M, L)
+    zroute, zexp = zcalls[0][1], zcalls[1][1]
+    zroute()
+    torch.cuda.synchronize()
+    zrows = (L["off"][1:] - L["off"][:-1]).cpu()
+    ms_route = time_kernel(torch, zroute, reps, flush)
+    ms_exp = time_kernel(torch, zexp, reps, flush)
+    zf = 6.0 * T * k * d * f
+    res["expert_fwd_zipf_router"] = {
+        "ms": round(ms_exp, 4), "TFLOPS": round(zf / ms_exp / 1e9, 1),
+        "frac_fp4_peak": round(zf / ms_exp / 1e9 / (peaks["bf16_sustained"] * 4.0), 4),
+        "route_permute_ms": round(ms_route, 4),
+        "rows_per_expert_padded": {"max": int(zrows.max()), "median": int(zrows.median()),
+                                   "min": int(zrows.min())}}
+    L["logits"] = saved
+    zroute = zexp = zcalls = None
+    layer_calls(M, L)[0][1]()  # routing of the uniform layer restored
+    torch.cuda.synchronize()
+    del zl
+
     # NVFP4 quantization of the layer input x, one pass (amax given) and two passes
     codes = torch.empty(T, d // 2, dtype=torch.uint8, device=dev)
     sc = torch.empty(T * d // 16, dtype=torch.uint8, device=dev)
@@ -462,27 +487,52 @@ def main():
     value = replica_value(flops, ms, world)
 
     # ---- end to end: host buffers, copies inside the timed region ----
-    stream = torch.cuda.current_stream()
+    # Every step copies its inputs from pinned host memory and its output back,
+    # as a serving loop would, with the copies of one step overlapping the
+    # compute of its neighbours: host-to-device copies, the layer and the
+    # device-to-host copy run on three streams over two sets of device
+    # buffers, ordered by events. The clock runs from before the first input
+    # copy to after the last output copy.
+    s_h2d, s_comp, s_d2h = torch.cuda.Stream(), torch.cuda.current_stream(), torch.cuda.Stream()
+    bufs = [{"x": L["x"], "logits": L["logits"], "out": L["out"]},
+            {"x": torch.empty_like(L["x"]), "logits": torch.empty_like(L["logits"]),
+             "out": torch.empty_like(L["out"])}]
+    ev = [{n: torch.cuda.Event() for n in ("h2d", "comp", "d2h")} for _ in range(2)]
     ea = torch.cuda.Event(enable_timing=True)
     eb = torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    ea.record()
-    for _ in range(args.steps):
-        L["x"].copy_(L["x_host"], non_blocking=True)
-        L["logits"].copy_(L["logits_host"], non_blocking=True)
+    ea.record(s_h2d)
+    for i in range(args.steps):
+        b, B = i % 2, bufs[i % 2]
+        with torch.cuda.stream(s_h2d):
+            if i >= 2:
+                s_h2d.wait_event(ev[b]["comp"])  # step i - 2 is done reading B
+            B["x"].copy_(L["x_host"], non_blocking=True)
+            B["logits"].copy_(L["logits_host"], non_blocking=True)
+            ev[b]["h2d"].record(s_h2d)
+        s_comp.wait_event(ev[b]["h2d"])
+        if i >= 2:
+            s_comp.wait_event(ev[b]["d2h"])  # step i - 2's output has left B
+        L["x"], L["logits"], L["out"] = B["x"], B["logits"], B["out"]
         for _, fn in calls:
             fn()
-        L["out_host"].copy_(L["out"], non_blocking=True)
-    eb.record()
+        ev[b]["comp"].record(s_comp)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(ev[b]["comp"])
+            L["out_host"].copy_(B["out"], non_blocking=True)
+            ev[b]["d2h"].record(s_d2h)
+    eb.record(s_d2h)
     torch.cuda.synchronize()
+    L["x"], L["logits"], L["out"] = bufs[0]["x"], bufs[0]["logits"], bufs[0]["out"]
+    del bufs
     clocks = sampler.stop()
     e2e_ms = max_over_ranks(ea.elapsed_time(eb) / args.steps, dist, dev)
     e2e = {"value": replica_value(flops, e2e_ms, world), "unit": "TFLOPS",
            "h2d_bytes_per_step": L["x_host"].numel() * 2 + L["logits_host"].numel() * 4,
-           "d2h_bytes_per_step": L["out_host"].numel() * 2, "ms_per_step": e2e_ms}
-    del stream
+           "d2h_bytes_per_step": L["out_host"].numel() * 2, "ms_per_step": e2e_ms,
+           "copies": "overlapped with compute across steps (3 streams, 2 buffer sets)"}
 
     fp4_peak = peaks["bf16_sustained"] * 4.0
     ex_ms = per_call["moe_expert_fwd"]
