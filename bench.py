@@ -281,6 +281,23 @@ def companions(M, synth, torch, dev, L, peaks, reps=10):
     ps8 = torch.empty(Rr, d // 32, dtype=torch.uint8, device=dev)
     gbs("rht32_mxfp8", lambda: M.rht32_quantize(pay, 11, M.FMT_MXFP8, pc8, ps8), Rr * d, 3.03125)
     del pay, pc8, ps8
+    # combine read straight from the RHT32 + NVFP4 payload of the layer's y
+    # (one inverse transform per token) against the bf16 combine of y
+    Ru = int(L["off"][-1])  # rows the layer wrote
+    yc = torch.empty(Ru, d // 2, dtype=torch.uint8, device=dev)
+    ys = torch.empty(Ru, d // 16, dtype=torch.uint8, device=dev)
+    yts = torch.empty(1, device=dev)
+    M.rht32_quantize(L["y"][:Ru], 11, M.FMT_NVFP4, yc, ys, yts)
+    cout = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    ms_rht = time_kernel(torch, lambda: M.moe_combine_rht(yc, ys, yts, M.FMT_NVFP4, 11, L["pos"],
+                                                          L["w"], cout), reps, flush)
+    ms_bf16 = time_kernel(torch, lambda: M.moe_combine(L["y"], L["pos"], L["w"], cout), reps, flush)
+    moved = T * k * (d // 2 + d // 16) + T * d * 2
+    res["combine_rht_nvfp4"] = {"ms": round(ms_rht, 4), "GB/s": round(moved / ms_rht / 1e6, 1),
+                                "frac_hbm": round(moved / ms_rht / 1e6 / hbm, 3),
+                                "bf16_combine_ms": round(ms_bf16, 4),
+                                "payload_bytes_vs_bf16": round((d // 2 + d // 16) / (2 * d), 4)}
+    del yc, ys, cout
     # MXFP8 backward operands on the permuted, per-expert padded layout
     off = L["off"].cpu().numpy()
     tok = L["tok"].cpu().numpy()

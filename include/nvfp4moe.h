@@ -104,12 +104,15 @@ const char *nvfp4moe_last_error(void);
  * identifier of the wait that ran out. Returns NVFP4MOE_ERR_TIMEOUT if set. */
 nvfp4moe_status nvfp4moe_device_error(int32_t *code);
 
-/* Exhaustive check of the hardware conversions the quantizers use against the
- * library's own encoders (which the test suite pins bit for bit to the CPU
- * reference): which = 0 checks cvt.rn.satfinite.e2m1x2.f32, which = 1
- * cvt.rn.satfinite.e4m3x2.f32, each over every finite fp32 input. The
- * mismatch count lands in *mismatches (device uint64, overwritten). Has no
- * counterpart on the pages; it guards the encoders on a new driver. */
+/* Exhaustive check of the hardware conversions the kernels use against the
+ * library's own encoders and decoders (which the test suite pins bit for bit
+ * to the CPU reference): which = 0 checks cvt.rn.satfinite.e2m1x2.f32 and
+ * which = 1 cvt.rn.satfinite.e4m3x2.f32, each over every finite fp32 input;
+ * which = 2 checks the decode cvt.rn.f16x2.e2m1x2 over all 256 code pairs
+ * and which = 3 cvt.rn.f16x2.e4m3x2 over all 65536 code pairs (the NaN codes
+ * 0x7F / 0xFF excepted: the encoders saturate and never write them). The mismatch
+ * count lands in *mismatches (device uint64, overwritten). Has no counterpart
+ * on the pages; it guards the conversions on a new driver. */
 nvfp4moe_status nvfp4moe_selftest(int which, unsigned long long *mismatches,
                                   nvfp4moe_stream_t stream);
 
@@ -275,6 +278,24 @@ nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const fl
 nvfp4moe_status moe_combine(const uint16_t *y, const int32_t *pos, const float *topk_w,
                             int64_t T, int32_t k, int64_t d, uint16_t *out,
                             nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Combine straight from the RHT32-quantized payload (aicoder.com 'Key
+ * Takeaways' and 'Architecture highlights': the expert-parallel combine
+ * traffic travels block-scaled after a 32-point random Hadamard transform).
+ * out[t] = bf16( RHT32^-1( sum_{j=0..k-1} topk_w[t,j] * v[pos[t,j]] ) ) per
+ * 32-block: the dequantized payload rows v are summed in fp32 in slot order
+ * with fused multiply-adds, then transformed once per token (the transform is
+ * linear, so this is the combine of the inverse-transformed rows).
+ * codes / scales / ts: a payload as written by rht32_quantize with the same
+ * sign_seed and fmt, ROWMAJOR scales: NVFP4 codes [* x d/2], scales
+ * [* x d/16], ts one device fp32; MXFP8 codes [* x d], scales [* x d/32], ts
+ * unused (may be NULL). pos, topk_w [T x k]; out bf16 [T x d]. d % 32 == 0.
+ * Caller owns all buffers; nothing is allocated. */
+nvfp4moe_status moe_combine_rht(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                int fmt, uint64_t sign_seed, const int32_t *pos,
+                                const float *topk_w, int64_t T, int32_t k, int64_t d,
+                                uint16_t *out, nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Grouped block-scaled GEMMs on the tcgen05 tensor cores.

@@ -131,7 +131,7 @@ nvfp4moe_status nvfp4moe_device_error(int32_t *code) {
 
 nvfp4moe_status nvfp4moe_selftest(int which, unsigned long long *mismatches,
                                   nvfp4moe_stream_t stream) {
-    NEED(which == 0 || which == 1, NVFP4MOE_ERR_INVALID_ARG, "nvfp4moe_selftest: which is 0 or 1");
+    NEED(which >= 0 && which <= 3, NVFP4MOE_ERR_INVALID_ARG, "nvfp4moe_selftest: which is 0..3");
     NEED_PTR4(mismatches);
     return after_launch(launch_selftest(which, mismatches, (cudaStream_t)stream),
                         "nvfp4moe_selftest");
@@ -372,6 +372,23 @@ nvfp4moe_status moe_combine(const uint16_t *y, const int32_t *pos, const float *
     }
     return after_launch(launch_combine(y, pos, topk_w, T, k, d, out, (cudaStream_t)stream),
                         "moe_combine");
+}
+
+nvfp4moe_status moe_combine_rht(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                                int fmt, uint64_t sign_seed, const int32_t *pos,
+                                const float *topk_w, int64_t T, int32_t k, int64_t d,
+                                uint16_t *out, nvfp4moe_stream_t stream) {
+    NEED(T >= 0 && k >= 1 && d > 0, NVFP4MOE_ERR_INVALID_ARG, "moe_combine_rht: sizes");
+    NEED(fmt == NVFP4MOE_FMT_NVFP4 || fmt == NVFP4MOE_FMT_MXFP8, NVFP4MOE_ERR_INVALID_ARG,
+         "moe_combine_rht: bad fmt");
+    NEED(d % 32 == 0, NVFP4MOE_ERR_SHAPE, "moe_combine_rht: d %% 32 == 0 required");
+    if (T > 0) {
+        NEED_PTR(codes); NEED_PTR(scales); NEED_PTR4(pos); NEED_PTR4(topk_w); NEED_PTR(out);
+        if (fmt == NVFP4MOE_FMT_NVFP4) NEED_PTR4(ts);
+    }
+    return after_launch(launch_combine_rht(codes, scales, ts, fmt, sign_seed, pos, topk_w, T, k, d,
+                                           out, (cudaStream_t)stream),
+                        "moe_combine_rht");
 }
 
 nvfp4moe_status nvfp4_grouped_gemm(const uint8_t *a, const uint8_t *a_sc, const float *a_ts,

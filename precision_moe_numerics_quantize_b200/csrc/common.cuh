@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "../../include/nvfp4moe.h"
@@ -48,6 +49,21 @@ NV_DEV uint32_t f32_to_bf16_bits(float f) {
     if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return 0x7FC0u;
     u += 0x7FFFu + ((u >> 16) & 1u);
     return u >> 16;
+}
+
+// Hardware decodes of packed low-precision pairs to two fp32 values: the low
+// nibble / byte lands in .x. Exact (every E2M1 and E4M3 value is an fp16).
+NV_DEV float2 e2m1x2_decode_hw(uint32_t byte) {
+    uint32_t h;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u16 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h)
+        : "h"((uint16_t)byte));
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+}
+NV_DEV float2 e4m3x2_decode_hw(uint32_t two_bytes) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)two_bytes));
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h));
 }
 
 // Two floats to a bf16 pair, round to nearest even (lo in bits 0..15).

@@ -475,6 +475,71 @@ __global__ void __launch_bounds__(256) rht32_dequant_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Combine straight from the RHT32-quantized payload: per token and 32-block,
+// sum_j w_j * dequant(v_j) in fp32 (slot order, fused multiply-adds), then one
+// inverse transform (butterflies, times c, sign flip) -> bf16. The transform
+// is linear, so this equals combining the inverse-transformed rows, with one
+// transform per token instead of k.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) combine_rht_kernel(
+    const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+    const float *__restrict__ ts_p, int fmt, uint64_t sign_seed, const int32_t *__restrict__ pos,
+    const float *__restrict__ w, int64_t T, int32_t k, int64_t d, uint16_t *__restrict__ out) {
+    const uint32_t signs = rht_signs_dev(sign_seed);
+    const int64_t G = d / 32;
+    const float ts = (fmt == NVFP4MOE_FMT_NVFP4) ? *ts_p : 1.0f;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < T * G;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / G, b = i - t * G;
+        float acc[32];
+#pragma unroll
+        for (int m = 0; m < 32; ++m) acc[m] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int64_t r = pos[t * k + j];
+            const float wj = w[t * k + j];
+            if (fmt == NVFP4MOE_FMT_NVFP4) {
+                const uint4 q = __ldg(reinterpret_cast<const uint4 *>(codes + r * (d / 2) + b * 16));
+                const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+                const uint16_t sc = __ldg(reinterpret_cast<const uint16_t *>(scales + r * (d / 16) + 2 * b));
+                // w_j * (block scale * tensor scale): one coefficient per 16 values
+                const float c0 = __fmul_rn(wj, __fmul_rn(e4m3_decode(sc & 0xFFu), ts));
+                const float c1 = __fmul_rn(wj, __fmul_rn(e4m3_decode(sc >> 8), ts));
+#pragma unroll
+                for (int m = 0; m < 32; m += 2) {
+                    const float2 v = e2m1x2_decode_hw((qs[m >> 3] >> (4 * (m & 7))) & 0xFFu);
+                    const float cm = m < 16 ? c0 : c1;
+                    acc[m] = fmaf(cm, v.x, acc[m]);
+                    acc[m + 1] = fmaf(cm, v.y, acc[m + 1]);
+                }
+            } else {
+                const float cj = scale_pow2(wj, 127 - (int)__ldg(scales + r * G + b));  // w_j * 2^(e - 127)
+                const uint4 *cq = reinterpret_cast<const uint4 *>(codes + r * d + b * 32);
+                const uint4 q0 = __ldg(cq), q1 = __ldg(cq + 1);
+                const uint32_t qs[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                for (int m = 0; m < 32; m += 2) {
+                    const float2 v = e4m3x2_decode_hw((qs[m >> 2] >> (8 * (m & 3))) & 0xFFFFu);
+                    acc[m] = fmaf(cj, v.x, acc[m]);
+                    acc[m + 1] = fmaf(cj, v.y, acc[m + 1]);
+                }
+            }
+        }
+        fwht32(acc);
+        uint32_t pk[16];
+#pragma unroll
+        for (int m = 0; m < 32; m += 2) {
+            float u0 = __fmul_rn(acc[m], RHT_C), u1 = __fmul_rn(acc[m + 1], RHT_C);
+            if ((signs >> m) & 1u) u0 = -u0;
+            if ((signs >> (m + 1)) & 1u) u1 = -u1;
+            pk[m >> 1] = f32_to_bf16_bits(u0) | (f32_to_bf16_bits(u1) << 16);
+        }
+        uint4 *op = reinterpret_cast<uint4 *>(out + t * d + b * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) op[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
 static int grid_for(int64_t work, int per_block = 256) {
@@ -602,6 +667,15 @@ cudaError_t launch_rht32_dequantize(const uint8_t *codes, const uint8_t *scales,
     return cudaGetLastError();
 }
 
+cudaError_t launch_combine_rht(const uint8_t *codes, const uint8_t *scales, const float *ts, int fmt,
+                               uint64_t sign_seed, const int32_t *pos, const float *w, int64_t T,
+                               int32_t k, int64_t d, uint16_t *out, cudaStream_t s) {
+    if (T * d == 0) return cudaSuccess;
+    combine_rht_kernel<<<grid_for(T * (d / 32)), 256, 0, s>>>(codes, scales, ts, fmt, sign_seed, pos,
+                                                              w, T, k, d, out);
+    return cudaGetLastError();
+}
+
 // grouped NVFP4 quantization of the expert activations h with per-expert
 // tensor scales: rows [off[e], off[e+1]) use amax[e]; ts[e] = amax[e] / 2688.
 __global__ void __launch_bounds__(256) nvfp4_quant_grouped_kernel(
@@ -651,7 +725,32 @@ cudaError_t launch_nvfp4_quant_grouped(const uint16_t *x, int64_t rows_alloc, in
 __global__ void __launch_bounds__(256) selftest_cvt_kernel(int which,
                                                            unsigned long long *mismatches) {
     unsigned long long bad = 0;
-    const uint64_t groups = 1ull << 29;  // 8 consecutive bit patterns per group
+    // which 2 / 3: the decodes cvt.rn.f16x2.e2m1x2 / .e4m3x2 over every packed
+    // pair against the software decoders, bit for bit
+    if (which >= 2) {
+        const uint32_t n = which == 2 ? 256u : 65536u;
+        for (uint32_t c = blockIdx.x * blockDim.x + threadIdx.x; c < n; c += gridDim.x * blockDim.x) {
+            float2 hw;
+            float lo, hi;
+            if (which == 2) {
+                hw = e2m1x2_decode_hw(c);
+                lo = e2m1_decode(c & 15u);
+                hi = e2m1_decode(c >> 4);
+            } else {
+                hw = e4m3x2_decode_hw(c);
+                lo = e4m3_decode(c & 0xFFu);
+                hi = e4m3_decode(c >> 8);
+            }
+            // E4M3 codes 0x7F / 0xFF are NaN; the library's encoders saturate
+            // and never write them, and its decoder is defined on the others
+            const bool skip_lo = which == 3 && (c & 0x7Fu) == 0x7Fu;
+            const bool skip_hi = which == 3 && ((c >> 8) & 0x7Fu) == 0x7Fu;
+            const bool ok_lo = skip_lo || __float_as_uint(lo) == __float_as_uint(hw.x);
+            const bool ok_hi = skip_hi || __float_as_uint(hi) == __float_as_uint(hw.y);
+            bad += (ok_lo ? 0 : 1) + (ok_hi ? 0 : 1);
+        }
+    }
+    const uint64_t groups = which >= 2 ? 0 : 1ull << 29;  // 8 consecutive bit patterns per group
     for (uint64_t g = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; g < groups;
          g += (uint64_t)gridDim.x * blockDim.x) {
         const uint32_t base = (uint32_t)(g << 3);

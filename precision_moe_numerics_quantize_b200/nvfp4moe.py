@@ -58,6 +58,7 @@ _SIGS = {
     "moe_expert_fwd": (C.c_int, [_P, _P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                  _P, _P, _P, _P, _P, _I64, _P]),
     "moe_combine": (C.c_int, [_P, _P, _P, _I64, _I32, _I64, _P, _P]),
+    "moe_combine_rht": (C.c_int, [_P, _P, _P, _I, _U64, _P, _P, _I64, _I32, _I64, _P, _P]),
     "nvfp4_grouped_gemm": (C.c_int, [_P, _P, _P, _I32, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P,
                                      _I, _P]),
     "mxfp8_grouped_gemm": (C.c_int, [_P, _P, _P, _P, _P, _I32, _I, _I64, _I64, _I64, _P, _I, _P]),
@@ -211,6 +212,15 @@ def moe_combine(y, pos, topk_w, out, stream=None):
     d = out.shape[1]
     _check("moe_combine", lib().moe_combine(
         _ptr(y), _ptr(pos), _ptr(topk_w), T, k, d, _ptr(out), _stream(stream)))
+
+
+def moe_combine_rht(codes, scales, ts, fmt, sign_seed, pos, topk_w, out, stream=None):
+    """Combine from an RHT32-quantized payload (as written by rht32_quantize)."""
+    T, k = pos.shape
+    d = out.shape[1]
+    _check("moe_combine_rht", lib().moe_combine_rht(
+        _ptr(codes), _ptr(scales), _ptr(ts), fmt, sign_seed, _ptr(pos), _ptr(topk_w), T, k, d,
+        _ptr(out), _stream(stream)))
 
 
 def nvfp4_grouped_gemm(a, a_sc, a_ts, a_ts_stride, b, b_sc, b_ts, group_off, G, R, N, K, c,
