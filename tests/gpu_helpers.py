@@ -33,6 +33,14 @@ def mma_index(rows: int, nsc: int) -> np.ndarray:
     return chunk * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (c % 4)
 
 
+def mma_rows_to_rowmajor(flat: np.ndarray, rows_idx: np.ndarray, nsc: int) -> np.ndarray:
+    """Row-major scales of the listed rows of an MMA-layout scale buffer."""
+    r = np.asarray(rows_idx, np.int64)[:, None]
+    c = np.arange(nsc)[None, :]
+    chunk = (r // 128) * (nsc // 4) + c // 4
+    return np.asarray(flat).reshape(-1)[chunk * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (c % 4)]
+
+
 def mma_to_rowmajor(flat: np.ndarray, rows: int, nsc: int) -> np.ndarray:
     return np.asarray(flat).reshape(-1)[mma_index(rows, nsc)]
 
