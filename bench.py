@@ -37,10 +37,10 @@ if ROOT not in sys.path:
 
 METRIC = "NVFP4 expert-FFN fwd TFLOPS (% of B200 FP4 peak); quantizer HBM GB/s"
 # dram__bytes_read.sum + dram__bytes_write.sum of moe_expert_fwd's three
-# kernels (GEMM1 + SwiGLU 5.745 GB, requantize 0.952 GB, GEMM2 3.66 GB) per
-# call of the full-size layer, from a 1-pass ncu capture of the CTA-pair GEMM
-# (summary under profiles/). Set back to None when those kernels change.
-EXPERT_FWD_DRAM_BYTES = 10.357e9
+# kernels (GEMM1 + SwiGLU 5.625 GB, requantize 0.953 GB, GEMM2 3.667 GB) per
+# call of the full-size layer, from a 1-pass ncu capture of the current
+# kernels (summary under profiles/). Set back to None when they change.
+EXPERT_FWD_DRAM_BYTES = 10.245e9
 
 
 def load_peaks():
@@ -558,7 +558,7 @@ def main():
                 "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
                 "traffic": EXPERT_FWD_DRAM_BYTES if args.workload == "full_moe" else None,
                 "traffic_frac_hbm": (round(EXPERT_FWD_DRAM_BYTES / (ex_ms * 1e-3) / (peaks["hbm_gbs"] * 1e9), 4)
-                                     if args.workload == "full_moe" else None),
+                                     if args.workload == "full_moe" and EXPERT_FWD_DRAM_BYTES else None),
                 "kernel": "moe_expert_fwd (grouped GEMM1+SwiGLU+amax, requantize, grouped GEMM2)",
                 "peak_source": f"{peaks['source']} bf16 sustained x 4 (nominal FP4:BF16 ratio)",
                 "weights_hbm_floor_ms": round(0.5625 * 3 * d * f * E / (peaks["hbm_gbs"] * 1e6), 3)}

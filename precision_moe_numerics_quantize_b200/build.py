@@ -20,6 +20,11 @@ FLAGS = [
 ]
 
 
+# Compiled as whole programs (no relocatable device code): ptxas ignores
+# setmaxnreg in relocatable code, and the GEMM's register split needs it.
+WHOLE_PROGRAM = {"gemm.cu"}
+
+
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -41,7 +46,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(build_dir, exist_ok=True)
     for src in sources():
         obj = os.path.join(build_dir, os.path.basename(src) + ".o")
-        cmd = [NVCC, *FLAGS, "-dc", src, "-o", obj]
+        mode = "-c" if os.path.basename(src) in WHOLE_PROGRAM else "-dc"
+        cmd = [NVCC, *FLAGS, mode, src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.check_call(cmd)

@@ -23,7 +23,9 @@ nvfp4moe_status cuda_status(cudaError_t e, const char *what);
 
 // Device error word: a kernel whose bounded wait ran out stores the id of the
 // wait here (first writer wins) and returns early.
+#ifndef NVFP4MOE_WHOLE_PROGRAM
 extern __device__ int32_t g_device_error;
+#endif
 
 enum WaitId : int32_t {
     WAIT_NONE = 0,
@@ -34,7 +36,7 @@ enum WaitId : int32_t {
     WAIT_GEMM_DRAIN = 5,
     WAIT_GEMM_SF_SLOT = 6,
     WAIT_GEMM_SF_FULL = 7,
-    WAIT_GEMM_SF_READY = 8,
+    WAIT_GEMM_SF_FREE = 8,
 };
 
 // ---------------------------------------------------------------------------
@@ -359,15 +361,15 @@ NV_DEV uint64_t globaltimer_ns() {
 }
 
 // Wait for the phase with the given parity to complete, giving up after about
-// two seconds: on timeout the wait id goes to the device error word and the
-// caller returns false so the kernel can wind down instead of hanging.
-NV_DEV bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int32_t wait_id) {
+// two seconds: on timeout the wait id goes to the device error word `err` and
+// the caller returns false so the kernel can wind down instead of hanging.
+NV_DEV bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int32_t *err, int32_t wait_id) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer_ns() - t0 > 2000000000ull) {
-            atomicCAS(&g_device_error, 0, wait_id);
+            atomicCAS(err, 0, wait_id);
             return false;
         }
     }
@@ -565,6 +567,11 @@ NV_DEV void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
                      taddr),
                  "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
                  "r"(r[7])
+                 : "memory");
+}
+NV_DEV void tmem_st_32x32b_x4(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3)
                  : "memory");
 }
 NV_DEV void tmem_st_32x32b_x1(uint32_t taddr, uint32_t r) {

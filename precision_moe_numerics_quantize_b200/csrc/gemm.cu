@@ -73,6 +73,10 @@
 // the device error word and raises this CTA's abort flag; the CTA winds down
 // and the other CTA of the pair then runs out on its own waits. Both CTAs meet
 // at a final cluster barrier before TMEM is released.
+// Built as a whole program (not relocatable device code) so that ptxas
+// applies the setmaxnreg register split; the device error word is reached
+// through a pointer in the kernel parameters.
+#define NVFP4MOE_WHOLE_PROGRAM 1
 #include "common.cuh"
 #include "quant.cuh"
 
@@ -92,19 +96,24 @@ constexpr int X_STAGE = 2 * X_KBLK;
 // (NVFP4: 4 chunks per k-block; MXFP8: 1)
 constexpr int SFX_CHUNKS = 8, SFX_STAGE = 2 * SFX_CHUNKS * 512;
 // scale warps come in SCALE_SETS sets of four taking turns by stage; the
-// epilogue's two warps per lane quarter follow them
+// epilogue's warps follow them.
 // Warpgroups: 0 = producer, MMA issuer and two idle warps; 1 = scale warps
 // (SCALE_SETS sets of four); then the epilogue, three warps per TMEM lane
 // quarter, each owning at most two 32-column blocks of a tile of up to
-// MAX_N = 192 columns. setmaxnreg moves registers from warpgroup 0 to the
-// epilogue: 128 x 48 + 128 x 96 + 384 x 120 = 64512 <= 640 x 102.
+// MAX_N = 192 columns. The kernel launches with 96 registers a thread
+// (640 x 96 = 61440); setmaxnreg moves some from warpgroup 0 to the
+// epilogue within that budget.
 constexpr int SCALE_SETS = 1;
 constexpr int SCALE_WARP0 = 4, EPI_WARP0 = SCALE_WARP0 + 4 * SCALE_SETS;
 constexpr int EPI_PER_QUARTER = 3, EPI_WARPS = 4 * EPI_PER_QUARTER;
 constexpr int NUM_THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
-constexpr uint32_t REGS_CONTROL = 48, REGS_EPILOGUE = 120;
+// Measured on the full-size expert FFN (same box): 56 / 96 / 104 took
+// 3.44 ms, no split 3.45 ms, 64 / 88 / 104 3.50 ms, 48 / 88 / 112 3.71 ms
+// (the MMA and producer loops spill at 48).
+constexpr uint32_t REGS_LAUNCH = 96, REGS_CONTROL = 56, REGS_EPILOGUE = 104;
 static_assert(NUM_THREADS == 640, "register split below assumes 20 warps");
-static_assert(128 * REGS_CONTROL + 128 * 96 + 32 * EPI_WARPS * REGS_EPILOGUE <= 65536, "register split");
+static_assert(128 * REGS_CONTROL + 128 * REGS_LAUNCH + 32 * EPI_WARPS * REGS_EPILOGUE <= NUM_THREADS * REGS_LAUNCH,
+              "setmaxnreg split exceeds the registers the block launches with");
 constexpr int MAX_GROUPS = 1024;
 constexpr uint32_t TMEM_COLS = 512, TMEM_SF = MAX_N, SF_KB_COLS = 48, SF_SLOT_COLS = 96;
 
@@ -151,6 +160,7 @@ struct Params {
     int32_t wtiles;        // 256-row W tiles per group (SwiGLU: f / 128)
     void *c;
     float *amax;
+    int32_t *err;  // device error word
 };
 
 struct Tile {
@@ -225,15 +235,15 @@ __device__ __forceinline__ Tile cursor_tile(const Params &p, const Cursor &c) {
 
 // Bounded wait that also gives up when another role of this CTA raised the
 // abort flag.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int32_t *abort_flag, int32_t id) {
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *abort_flag,
+                                              int32_t *err, int32_t id) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > 2000000000ull) {
-            atomicCAS(&g_device_error, 0, id);
+            atomicCAS(err, 0, id);
             *abort_flag = 1;
             return false;
         }
@@ -349,7 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int xcr = (int)((T.x_row + T.n - 1) / 128 - xa) + 1;
                 for (int kb0 = 0; kb0 < T.kt; kb0 += 2) {
                     const int nkb = T.kt - kb0 >= 2 ? 2 : 1;
-                    if (!wait_or_abort(&empty[s], phase ^ 1u, abort_flag, WAIT_GEMM_EMPTY)) {
+                    if (!wait_or_abort(&empty[s], phase ^ 1u, abort_flag, p.err, WAIT_GEMM_EMPTY)) {
                         ok = false;
                         break;
                     }
@@ -384,7 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
         }
     } else if (warp >= SCALE_WARP0 && warp < EPI_WARP0) {
-        // ======================= scale warps =======================
+        // ======================= scale warps (launch registers) =======================
         // In a 512-byte scale chunk the word (4 scales) of row r0 + 32 r1 sits
         // at byte r0 * 16 + r1 * 4, so lane r0 reads 16 contiguous bytes per X
         // chunk (the words of X rows r0 + 32 j) and one word of each W chunk:
@@ -442,8 +452,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // the stage's bytes landed (first CTA: operands and X scales on
             // `full`; other CTA: its X scales on `sf_loaded`); the producer
             // only loaded them after the MMAs that last read slot s were done
-            const bool ok = rank == 0 ? wait_or_abort(&full[sb], par, abort_flag, WAIT_GEMM_FULL)
-                                      : wait_or_abort(&sf_loaded[sb], par, abort_flag, WAIT_GEMM_SF_SLOT);
+            const bool ok = rank == 0 ? wait_or_abort(&full[sb], par, abort_flag, p.err, WAIT_GEMM_FULL)
+                                      : wait_or_abort(&sf_loaded[sb], par, abort_flag, p.err, WAIT_GEMM_SF_SLOT);
             if (!ok) return false;
             tc_fence_after();
             const int nkb = T.kt - st.kb0 >= 2 ? 2 : 1;
@@ -543,14 +553,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                  cursor_next(gtab, G, npairs32, c)) {
                 const Tile T = cursor_tile(p, c);
                 if (T.kt == 0) continue;
-                if (!wait_or_abort(acc_empty, acc_phase ^ 1u, abort_flag, WAIT_GEMM_ACC_EMPTY)) break;
+                if (!wait_or_abort(acc_empty, acc_phase ^ 1u, abort_flag, p.err, WAIT_GEMM_ACC_EMPTY)) break;
                 tc_fence_after();
                 const uint32_t idesc4 = idesc_nvf4(T.n);
                 for (int kb0 = 0; kb0 < T.kt; kb0 += 2) {
                     const int nkb = T.kt - kb0 >= 2 ? 2 : 1;
                     // the scale warps arrive once the stage's scales are in
                     // TMEM and (first CTA) its operands in shared memory
-                    if (!wait_or_abort(&sf_full[s], phase, abort_flag, WAIT_GEMM_SF_FULL)) {
+                    if (!wait_or_abort(&sf_full[s], phase, abort_flag, p.err, WAIT_GEMM_SF_FULL)) {
                         ok = false;
                         break;
                     }
@@ -606,7 +616,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int nb = max(0, min(2, T.n / 32 - b0));
             const int64_t row0 = T.out_row + 32 * b0;  // output row of the first column
             if (have_acc) {
-                if (!wait_or_abort(acc_full, acc_phase, abort_flag, WAIT_GEMM_ACC_FULL)) break;
+                if (!wait_or_abort(acc_full, acc_phase, abort_flag, p.err, WAIT_GEMM_ACC_FULL)) break;
                 tc_fence_after();
             }
             uint32_t va[32], vb[32];
@@ -806,6 +816,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     p.wtiles = (int32_t)(swiglu ? p.f_out / 128 : a.N / 256);
     p.c = a.c;
     p.amax = a.amax;
+    p.err = device_error_word();
+    if (!p.err) return cudaErrorInvalidSymbol;
     // contraction bytes per row and scale chunks per 128-row block
     const int64_t kbytes = nvf4 ? a.a_cols / 2 : a.a_cols;
     p.x_nkc = nvf4 ? a.a_cols / 64 : a.a_cols / 128;
@@ -824,6 +836,13 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
         cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
         if (e != cudaSuccess) return e;
+        // setmaxnreg only redistributes the registers the block launched
+        // with: a build that gave the kernel fewer than REGS_LAUNCH would
+        // leave the epilogue's increase waiting forever
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, grouped_gemm_pair_kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs < (int)REGS_LAUNCH) return cudaErrorInvalidConfiguration;
         attr_set = true;
     }
     grouped_gemm_pair_kernel<<<pair_grid(), NUM_THREADS, SMEM_ALLOC, s>>>(mw, mx32, mx64, p);

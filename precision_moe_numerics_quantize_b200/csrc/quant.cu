@@ -14,6 +14,19 @@ namespace nvfp4moe {
 
 __device__ int32_t g_device_error = 0;
 
+int32_t *device_error_word() {
+    constexpr int kMaxDevices = 64;
+    static int32_t *addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int32_t *>(p);
+    }
+    return addr[dev];
+}
+
 // ---------------------------------------------------------------------------
 // amax of a bf16 tensor. *amax must be zero before the launch.
 // ---------------------------------------------------------------------------

@@ -71,6 +71,10 @@ struct GemmArgs {
     float *amax;      // SwiGLU: per-group amax of h
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s);
+// Device address of the device error word on the current device, for kernels
+// built as whole programs (they cannot name the variable itself); nullptr if
+// the runtime cannot resolve it.
+int32_t *device_error_word();
 cudaError_t launch_combine_rht(const uint8_t *codes, const uint8_t *scales, const float *ts, int fmt,
                                uint64_t sign_seed, const int32_t *pos, const float *w, int64_t T,
                                int32_t k, int64_t d, uint16_t *out, cudaStream_t s);

@@ -127,12 +127,14 @@ def test_grouped_nvfp4_gemm_ragged_groups(dev, lib, orc):
 
 
 def test_grouped_nvfp4_gemm_tile_shapes(dev, lib, orc):
-    """Groups of 640, 128, 512 and 896 rows: token tiles of 192, 128 and 64
-    rows, tiles that start 64 rows into a 128-row scale block, and K = 768
-    (three 128-byte k-blocks: a full and a half pipeline stage); bf16 out."""
-    rows = [640, 128, 512, 896]
+    """Groups of 640, 128, 512, 896, 384, 1152 and 768 rows: token tiles of
+    384 (MMAs of N = 256 and 128 on one W stage), 320 (256 + 64), 256 and 128
+    rows, tiles that start 64 rows into a 128-row scale block and span four
+    scale chunk rows, and K = 768 (three 128-byte k-blocks: the third reuses
+    the TMEM scale slot of the first); bf16 out."""
+    rows = [640, 128, 512, 896, 384, 1152, 768]
     off = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
-    R, K, N, G = int(off[-1]), 768, 256, 4
+    R, K, N, G = int(off[-1]), 768, 256, len(rows)
     A = _f32(synth.rows_np(7, synth.TAG_A, 0, R, K, 1.0))
     a_parts, a_sc, a_ts, Ad = [], [], [], np.zeros((R, K))
     for g in range(G):
@@ -187,10 +189,11 @@ def test_mxfp8_gemm_group_m(dev, lib, orc):
         _check_f32(got[sl], orc.gemm_f64(Ad[sl], Bd[g]), orc.gemm_f64(np.abs(Ad[sl]), np.abs(Bd[g])))
 
 
-@pytest.mark.parametrize("M", [256, 640])
+@pytest.mark.parametrize("M", [256, 384, 640])
 def test_mxfp8_gemm_group_k(dev, lib, orc, M):
     """Weight-gradient shape: C_g = A[:, off_g:off_g+1] . B[:, off_g:off_g+1]^T with an empty
-    group; M = 640 output rows give token-side tiles of 192 and 64 rows."""
+    group; M = 384 output rows make one token-side tile of two MMAs (N = 256 and 128),
+    M = 640 two tiles of 320 rows, the second starting 64 rows into a scale block."""
     seg = [256, 0, 128, 384]
     off = np.concatenate([[0], np.cumsum(seg)]).astype(np.int32)
     N, Kt, G = 256, int(off[-1]), 4
