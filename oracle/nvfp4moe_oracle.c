@@ -702,6 +702,68 @@ ORACLE_API void oracle_expert_ffn(const uint8_t *xq, const uint8_t *xq_sc, float
     free(A); free(H); free(B2); free(Hs); free(Y);
 }
 
+/* Dequantize an MXFP8 matrix (row-major E8M0 scales, blocks of 32 along
+ * columns) to fp64. */
+static void mxfp8_to_f64(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                         double *out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = oracle_e4m3_decode(codes[r * cols + c]) *
+                                ldexp(1.0, (int)scales[r * (cols / 32) + c / 32] - 127);
+}
+
+/*
+ * READING ([P2] "Architecture highlights": the last 16.6% of layers stay in
+ * MXFP8): the same expert forward as oracle_expert_ffn with every operand in
+ * MXFP8 instead of NVFP4: E4M3 codes with one E8M0 scale per 32 consecutive
+ * elements of a row, rounded to nearest-even (stochastic rounding is for the
+ * gradients), no tensor scale.
+ *   gu = dq(xq) * dq(W1_e)^T                (fp64)
+ *   h  = bf16(silu(g) * u)
+ *   hq = MXFP8(h) along rows, round-to-nearest-even
+ *   y  = bf16(dq(hq) * dq(W2_e)^T)
+ * xq: n x d codes + n x d/32 scales, W1: 2f x d, W2: d x f (row-major scales).
+ * Outputs h_bits [n x f], hq [n x f], hq_sc [n x f/32], y_bits [n_out or n
+ * rows x d]; rows_out as in oracle_expert_ffn.
+ */
+ORACLE_API void oracle_expert_ffn_mxfp8(const uint8_t *xq, const uint8_t *xq_sc, int64_t n,
+                                        int64_t d, int64_t f, const uint8_t *w1,
+                                        const uint8_t *w1_sc, const uint8_t *w2,
+                                        const uint8_t *w2_sc, const int32_t *rows_out,
+                                        int64_t n_out, uint16_t *h_bits, uint8_t *hq,
+                                        uint8_t *hq_sc, uint16_t *y_bits) {
+    double *A = (double *)malloc(sizeof(double) * (size_t)(n * d));
+    double *B1 = (double *)malloc(sizeof(double) * (size_t)(2 * f * d));
+    double *GU = (double *)malloc(sizeof(double) * (size_t)(n * 2 * f));
+    mxfp8_to_f64(xq, xq_sc, n, d, A);
+    mxfp8_to_f64(w1, w1_sc, 2 * f, d, B1);
+    oracle_gemm_f64(A, B1, n, 2 * f, d, GU);
+    free(A);
+    free(B1);
+    float *hf = (float *)malloc(sizeof(float) * (size_t)(n * f));
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t c = 0; c < f; ++c) {
+            uint16_t hb = oracle_bf16_from_f64(swiglu(GU[r * 2 * f + c], GU[r * 2 * f + f + c]));
+            h_bits[r * f + c] = hb;
+            hf[r * f + c] = oracle_bf16_to_f32(hb);
+        }
+    free(GU);
+    oracle_mxfp8_quantize(hf, n, f, 0, NULL, 0, 0, 0, 0, hq, hq_sc);
+    free(hf);
+    double *H = (double *)malloc(sizeof(double) * (size_t)(n * f));
+    double *B2 = (double *)malloc(sizeof(double) * (size_t)(d * f));
+    mxfp8_to_f64(hq, hq_sc, n, f, H);
+    mxfp8_to_f64(w2, w2_sc, d, f, B2);
+    int64_t cnt = rows_out ? n_out : n;
+    double *Hs = (double *)malloc(sizeof(double) * (size_t)(cnt * f));
+    for (int64_t i = 0; i < cnt; ++i)
+        memcpy(Hs + i * f, H + (rows_out ? rows_out[i] : i) * f, sizeof(double) * (size_t)f);
+    double *Y = (double *)malloc(sizeof(double) * (size_t)(cnt * d));
+    oracle_gemm_f64(Hs, B2, cnt, d, f, Y);
+    for (int64_t i = 0; i < cnt * d; ++i) y_bits[i] = oracle_bf16_from_f64(Y[i]);
+    free(H); free(B2); free(Hs); free(Y);
+}
+
 /*
  * READING ([P2] "Key Takeaways": the combine step): out[t] = sum over slots j
  * of w[t, j] * y[pos[t, j]] in fp64, rounded once to bf16. y rows are bf16.

@@ -16,7 +16,7 @@ __all__ = [
     "nvfp4_to_f64", "philox4x32_10", "philox_word", "mxfp8_quantize", "mxfp8_dequantize",
     "rht_signs", "rht32_forward_f32", "rht32_inverse_f32", "rht32_f64", "rht32_quantize",
     "rht32_dequantize", "route", "permute", "gemm_f64", "swiglu", "expert_ffn", "combine",
-    "combine_f32", "combine_rht", "mxfp8_rpad",
+    "combine_f32", "combine_rht", "mxfp8_rpad", "expert_ffn_mxfp8",
 ]
 
 _lib = None
@@ -66,6 +66,8 @@ def _declare(L):
         "oracle_swiglu": (C.c_double, [C.c_double, C.c_double]),
         "oracle_expert_ffn": (None, [_P, _P, C.c_float, _I64, _I64, _I64, _P, _P, C.c_float, _P,
                                      _P, C.c_float, _P, _I64, _P, _P, _P, _P, _P]),
+        "oracle_expert_ffn_mxfp8": (None, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _I64,
+                                           _P, _P, _P, _P]),
         "oracle_combine": (None, [_P, _P, _P, _I64, _I32, _I64, _P]),
         "oracle_combine_f32": (None, [_P, _P, _P, _I64, _I32, _I64, _P]),
         "oracle_combine_rht": (None, [_P, _P, C.c_float, C.c_int, _U64, _P, _P, _I64, _I32,
@@ -341,6 +343,27 @@ def expert_ffn(xq, xq_sc, x_ts, w1, w1_sc, w1_ts, w2, w2_sc, w2_ts, rows_out=Non
                             0 if ro is None else len(ro), _p(h), _p(hq), _p(hq_sc), _p(h_ts),
                             _p(y))
     return {"h": h, "hq": hq, "hq_sc": hq_sc, "h_ts": np.float32(h_ts[0]), "y": y}
+
+
+def expert_ffn_mxfp8(xq, xq_sc, w1, w1_sc, w2, w2_sc, rows_out=None):
+    """One expert's forward with MXFP8 operands. xq [n, d] E4M3 codes with row-major E8M0
+    scales [n, d/32], W1 [2f, d], W2 [d, f] likewise. Returns dict with h (bf16 bits [n, f]),
+    hq [n, f], hq_sc [n, f/32], y (bf16 bits [len(rows_out) or n, d])."""
+    xq = _c(xq, np.uint8); xq_sc = _c(xq_sc, np.uint8)
+    w1 = _c(w1, np.uint8); w1_sc = _c(w1_sc, np.uint8)
+    w2 = _c(w2, np.uint8); w2_sc = _c(w2_sc, np.uint8)
+    n, d = xq.shape
+    f = w2.shape[1]
+    ro = None if rows_out is None else _c(rows_out, np.int32)
+    cnt = n if ro is None else len(ro)
+    h = np.zeros((n, f), np.uint16)
+    hq = np.zeros((n, f), np.uint8)
+    hq_sc = np.zeros((n, f // 32), np.uint8)
+    y = np.zeros((cnt, d), np.uint16)
+    lib().oracle_expert_ffn_mxfp8(_p(xq), _p(xq_sc), n, d, f, _p(w1), _p(w1_sc), _p(w2),
+                                  _p(w2_sc), _p(ro), 0 if ro is None else len(ro), _p(h), _p(hq),
+                                  _p(hq_sc), _p(y))
+    return {"h": h, "hq": hq, "hq_sc": hq_sc, "y": y}
 
 
 def combine(y_bits, pos, w):

@@ -107,6 +107,61 @@ def test_expert_ffn_matches_dense_reference(orc):
     assert np.all(np.abs(yv - y) <= np.abs(y) * 2.0 ** -8 + slack + 1e-30)
 
 
+def _mx_decode_torch(codes, scales):
+    """MXFP8 decoded with torch's float8_e4m3fn and numpy powers of two."""
+    v = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return v * np.repeat(np.ldexp(1.0, scales.astype(np.int64) - 127), 32, axis=1)
+
+
+def _mx_quantize_torch(x):
+    """MXFP8 with round-to-nearest-even along rows: the smallest k with
+    amax <= 448 * 2^k per 32-block, codes by torch's float8_e4m3fn cast."""
+    rows, cols = x.shape
+    blocks = x.astype(np.float64).reshape(rows, cols // 32, 32)
+    amax = np.abs(blocks).max(axis=2)
+    with np.errstate(divide="ignore"):
+        k = np.where(amax > 0, np.ceil(np.log2(amax / 448.0)), -127.0)
+    k = np.clip(k, -127, 127).astype(np.int64)
+    v = blocks * np.ldexp(1.0, -k)[:, :, None]
+    codes = torch.from_numpy(v.reshape(rows, cols)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return codes, (k + 127).astype(np.uint8)
+
+
+def test_expert_ffn_mxfp8_matches_dense_reference(orc):
+    """The MXFP8 expert forward at a tiny size against an independent dense
+    reference: operands decoded with torch's float8_e4m3fn, numpy matmul, torch
+    SwiGLU, h requantized by a torch cast, matmul."""
+    n, d, f = 16, 64, 64
+    x = synth.bf16_bits_to_f32(synth.rows_np(0, synth.TAG_X, 0, n, d, 1.0))
+    xq, xs = orc.mxfp8_quantize(x, axis=0, rounding=0)
+    W1 = synth.bf16_bits_to_f32(synth.expert_weight_np(1, synth.TAG_W1, 0, 2 * f, d))
+    W2 = synth.bf16_bits_to_f32(synth.expert_weight_np(1, synth.TAG_W2, 0, d, f))
+    w1q, w1s = orc.mxfp8_quantize(W1, axis=0, rounding=0)
+    w2q, w2s = orc.mxfp8_quantize(W2, axis=0, rounding=0)
+    r = orc.expert_ffn_mxfp8(xq, xs, w1q, w1s, w2q, w2s)
+    A = _mx_decode_torch(xq, xs)
+    B1 = _mx_decode_torch(w1q, w1s)
+    gu = A @ B1.T
+    g, u = gu[:, :f], gu[:, f:]
+    h = (torch.nn.functional.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
+    mag1 = np.abs(A) @ np.abs(B1).T
+    hv = synth.bf16_bits_to_f32(r["h"]).astype(np.float64)
+    slack = 1e-12 * (mag1[:, :f] * np.abs(u) + mag1[:, f:] * np.abs(g))
+    assert np.all(np.abs(hv - h) <= np.abs(h) * 2.0 ** -8 + slack + 1e-30)
+    hq, hs = _mx_quantize_torch(synth.bf16_bits_to_f32(r["h"]))
+    assert np.array_equal(hq, r["hq"]) and np.array_equal(hs, r["hq_sc"])
+    H = _mx_decode_torch(hq, hs)
+    B2 = _mx_decode_torch(w2q, w2s)
+    y = H @ B2.T
+    yv = synth.bf16_bits_to_f32(r["y"]).astype(np.float64)
+    slack = 1e-12 * (np.abs(H) @ np.abs(B2).T)
+    assert np.all(np.abs(yv - y) <= np.abs(y) * 2.0 ** -8 + slack + 1e-30)
+    # y rows requested one by one equal the full result
+    sel = np.array([3, 0, 11], np.int32)
+    assert np.array_equal(orc.expert_ffn_mxfp8(xq, xs, w1q, w1s, w2q, w2s, rows_out=sel)["y"],
+                          r["y"][sel])
+
+
 def test_single_expert_top1_is_dense_mlp(orc):
     """E = 1, k = 1, renormalized weights: the layer reduces to out = MLP(x)."""
     T, d, f = 24, 64, 32
