@@ -58,24 +58,77 @@ def load_peaks():
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, read while the timed work
+    runs. An NVML reader thread polls every 2 ms (read-only queries) and is
+    running before the constructor returns; without NVML, nvidia-smi polls
+    every 100 ms instead."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, dev_index):
         self.proc = None
-        self.lines = []
+        self.thread = None
+        self.samples = []  # (sm MHz, reason mask)
+        self.max_mhz = None
+        self.source = None
         try:
             import torch
             uuid = "GPU-" + str(torch.cuda.get_device_properties(dev_index).uuid)
+        except Exception:
+            return
+        try:
+            import threading
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+            get_reasons = getattr(N, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                N.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.done = threading.Event()
+            started = threading.Event()
+
+            def poll():
+                while not self.done.is_set():
+                    try:
+                        self.samples.append((float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)),
+                                             int(get_reasons(h))))
+                    except Exception:
+                        pass
+                    started.set()
+                    time.sleep(0.002)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            started.wait(2.0)
+            self.source = "nvml, 2 ms"
+            return
+        except Exception:
+            self.thread = None
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi, 100 ms"
         except Exception:
             self.proc = None
 
+    def _summary(self, mhz, mx, reasons):
+        if not mhz:
+            return None
+        loaded = [m for m in mhz if mx and m > 0.3 * mx] or mhz
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz), "source": self.source}
+
     def stop(self):
+        if self.thread is not None:
+            self.done.set()
+            self.thread.join(timeout=5)
+            reasons = {n for n, bit in self.REASONS for _, m in self.samples if m & bit}
+            return self._summary([c for c, _ in self.samples], self.max_mhz, reasons)
         if not self.proc:
             return None
         self.proc.terminate()
@@ -85,7 +138,7 @@ class ClockSampler:
             self.proc.kill()
             out = ""
         mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _ in self.REASONS]
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
@@ -98,11 +151,7 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        if not mhz:
-            return None
-        loaded = [m for m in mhz if mx and m > 0.3 * mx] or mhz
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(mhz)}
+        return self._summary(mhz, mx, reasons)
 
 
 # ---------------------------------------------------------------------------
@@ -344,8 +393,44 @@ def companions(M, synth, torch, dev, L, peaks, reps=10):
     res["mxfp8_wgrad_gemm"] = {"ms": round(ms, 4), "TFLOPS": round(flops / ms / 1e9, 1),
                                "frac_fp8_peak": round(flops / ms / 1e9 / fp8_peak, 3),
                                "note": "fp32 dW [E x d x f] written"}
-    del dW, dy, act, dyc0, dys0, dyc1, dys1, ac1, as1, w2c, w2s, flush_buf
+    del dW, dy, act, dyc0, dys0, dyc1, dys1, ac1, as1, w2c, w2s
     torch.cuda.empty_cache()
+    # The expert FFN forward in MXFP8 (the layers that stay in MXFP8): the same
+    # routed rows, x / W1 / W2 quantized along rows with round-to-nearest-even
+    R = L["R"]
+    tok_d = torch.from_numpy(tok).to(dev)
+    xp = L["x"][tok_d.clamp(min=0).long()]
+    xp[tok_d < 0] = 0
+    xq8 = torch.empty(R, d, dtype=torch.uint8, device=dev)
+    xs8 = torch.empty(R * d // 32, dtype=torch.uint8, device=dev)
+    M.mxfp8_quantize_sr(xp, xq8, xs8, axis=0, rounding=M.ROUND_RNE, layout=M.LAYOUT_MMA)
+    del xp
+
+    def mx_weights(tag, rows, cols):
+        c = torch.empty(E * rows, cols, dtype=torch.uint8, device=dev)
+        s = torch.empty(E * rows * cols // 32, dtype=torch.uint8, device=dev)
+        for e in range(E):
+            wb = synth.expert_weight_torch(1, tag, e, rows, cols, dev)
+            M.mxfp8_quantize_sr(wb, c[e * rows:(e + 1) * rows],
+                                s[e * rows * cols // 32:(e + 1) * rows * cols // 32], axis=0,
+                                rounding=M.ROUND_RNE, layout=M.LAYOUT_MMA)
+        return c, s
+
+    w1m, w1ms = mx_weights(synth.TAG_W1, 2 * f, d)
+    w2m, w2ms = mx_weights(synth.TAG_W2, d, f)
+    hq8 = torch.empty(R, f, dtype=torch.uint8, device=dev)
+    hs8 = torch.empty(R * f // 32, dtype=torch.uint8, device=dev)
+    ham = torch.empty(E, device=dev)
+    ms = time_kernel(torch, lambda: M.moe_expert_fwd_mxfp8(xq8, xs8, L["off"], E, d, f, w1m, w1ms,
+                                                           w2m, w2ms, L["h"], ham, hq8, hs8, L["y"],
+                                                           R), reps, flush)
+    ff = 6.0 * T * k * d * f
+    res["expert_fwd_mxfp8"] = {"ms": round(ms, 4), "TFLOPS": round(ff / ms / 1e9, 1),
+                               "frac_fp8_peak": round(ff / ms / 1e9 / fp8_peak, 3)}
+    del xq8, xs8, w1m, w1ms, w2m, w2ms, hq8, hs8, ham, flush_buf
+    torch.cuda.empty_cache()
+    layer_calls(M, L)[1][1]()  # the layer's own h and y restored
+    torch.cuda.synchronize()
     res["fp8_peak_tflops"] = fp8_peak
     return res
 

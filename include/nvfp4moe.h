@@ -270,6 +270,36 @@ nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const fl
                                nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Expert FFN forward in MXFP8 (aicoder.com 'Architecture highlights': the last
+ * 16.6% of layers stay in MXFP8). The same computation as moe_expert_fwd
+ * with every operand in MXFP8: E4M3 codes with one E8M0 scale per 32
+ * consecutive elements of a row, round-to-nearest-even, no tensor scale.
+ * For every expert e, rows [expert_off[e], expert_off[e+1]):
+ *   [g | u] = dq(xq) . dq(W1_e)^T in fp32 on the tensor cores,
+ *   h       = bf16(silu(g) * u),  h_amax[e] = max |h| over the expert's rows,
+ *   hq      = MXFP8(h) along rows (round-to-nearest-even),
+ *   y       = bf16(dq(hq) . dq(W2_e)^T).
+ * xq [R x d] E4M3 codes in the dispatch layout of moe_route_permute (expert
+ *   blocks starting at multiples of 128 rows, padding rows zero), xq_sc the
+ *   MMA layout of its [R x d/32] E8M0 scales (mxfp8_quantize, axis 0).
+ * w1 [E x 2f x d] codes, w1_sc MMA layout of the [E*2f x d] matrix; rows
+ *   0..f-1 of W1_e give g, rows f..2f-1 give u. w2 [E x d x f], w2_sc MMA
+ *   layout of [E*d x f]. (Quantize with mxfp8_quantize, axis 0, RNE.)
+ * Caller-provided intermediates (outputs too): h bf16 [R x f], h_amax fp32
+ *   [E], hq [R x f] codes, hq_sc MMA layout of [R x f/32]. Rows of h and hq
+ *   past expert_off[E] hold no meaning.
+ * y bf16 [R x d]. R = rows_alloc >= expert_off[E], R % 128 == 0.
+ * d % 256 == 0, f % 256 == 0, E <= 1024. Pointers 16-byte aligned (4 for
+ * expert_off and h_amax). Errors: NVFP4MOE_ERR_INVALID_ARG, _SHAPE, _ALIGN
+ * before any launch; NVFP4MOE_ERR_CUDA for a failed launch. */
+nvfp4moe_status moe_expert_fwd_mxfp8(const uint8_t *xq, const uint8_t *xq_sc,
+                                     const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
+                                     const uint8_t *w1, const uint8_t *w1_sc, const uint8_t *w2,
+                                     const uint8_t *w2_sc, uint16_t *h, float *h_amax,
+                                     uint8_t *hq, uint8_t *hq_sc, uint16_t *y, int64_t rows_alloc,
+                                     nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Weighted top-k combine (aicoder.com 'Key Takeaways': the combine step).
  * out[t] = bf16( sum_{j=0..k-1} topk_w[t,j] * y[pos[t,j]] ), fp32 accumulation
  * in slot order with fused multiply-adds; a gather, no atomics.

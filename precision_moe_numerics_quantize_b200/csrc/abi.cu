@@ -362,6 +362,45 @@ nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const fl
     return after_launch(cudaSuccess, "moe_expert_fwd");
 }
 
+nvfp4moe_status moe_expert_fwd_mxfp8(const uint8_t *xq, const uint8_t *xq_sc,
+                                     const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
+                                     const uint8_t *w1, const uint8_t *w1_sc, const uint8_t *w2,
+                                     const uint8_t *w2_sc, uint16_t *h, float *h_amax,
+                                     uint8_t *hq, uint8_t *hq_sc, uint16_t *y, int64_t rows_alloc,
+                                     nvfp4moe_stream_t stream) {
+    NEED(E >= 1 && E <= 1024, NVFP4MOE_ERR_INVALID_ARG, "moe_expert_fwd_mxfp8: 1 <= E <= 1024");
+    NEED(d > 0 && f > 0 && rows_alloc >= 0, NVFP4MOE_ERR_INVALID_ARG, "moe_expert_fwd_mxfp8: sizes");
+    NEED(d % 256 == 0 && f % 256 == 0 && rows_alloc % 128 == 0, NVFP4MOE_ERR_SHAPE,
+         "moe_expert_fwd_mxfp8: d %% 256, f %% 256 and rows_alloc %% 128 must be 0");
+    NEED_PTR(xq); NEED_PTR(xq_sc); NEED_PTR4(expert_off);
+    NEED_PTR(w1); NEED_PTR(w1_sc); NEED_PTR(w2); NEED_PTR(w2_sc);
+    NEED_PTR(h); NEED_PTR4(h_amax); NEED_PTR(hq); NEED_PTR(hq_sc); NEED_PTR(y);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(h_amax, 0, sizeof(float) * E, s);
+    if (e != cudaSuccess) return cuda_status(e, "moe_expert_fwd_mxfp8: memset");
+    GemmArgs g1{};
+    g1.kind = 1; g1.epi = EPI_SWIGLU_AMAX; g1.group_axis = NVFP4MOE_GROUP_M;
+    g1.a = xq; g1.a_sc = xq_sc; g1.b = w1; g1.b_sc = w1_sc;
+    g1.group_off = expert_off; g1.G = E;
+    g1.a_rows = rows_alloc; g1.a_cols = d; g1.N = 2 * f; g1.b_rows_per_group = 2 * f;
+    g1.c = h; g1.amax = h_amax;
+    if ((e = launch_grouped_gemm(g1, s)) != cudaSuccess)
+        return cuda_status(e, "moe_expert_fwd_mxfp8: gemm1");
+    // per-32-block scales need no expert-wide pass: one row-wise quantize of h
+    if ((e = launch_mxfp8_quantize(h, rows_alloc, f, f, 0, 0, 0, NVFP4MOE_ROUND_RNE, hq, hq_sc,
+                                   NVFP4MOE_LAYOUT_MMA, s)) != cudaSuccess)
+        return cuda_status(e, "moe_expert_fwd_mxfp8: requantize");
+    GemmArgs g2{};
+    g2.kind = 1; g2.epi = EPI_STORE_BF16; g2.group_axis = NVFP4MOE_GROUP_M;
+    g2.a = hq; g2.a_sc = hq_sc; g2.b = w2; g2.b_sc = w2_sc;
+    g2.group_off = expert_off; g2.G = E;
+    g2.a_rows = rows_alloc; g2.a_cols = f; g2.N = d; g2.b_rows_per_group = d;
+    g2.c = y;
+    if ((e = launch_grouped_gemm(g2, s)) != cudaSuccess)
+        return cuda_status(e, "moe_expert_fwd_mxfp8: gemm2");
+    return after_launch(cudaSuccess, "moe_expert_fwd_mxfp8");
+}
+
 nvfp4moe_status moe_combine(const uint16_t *y, const int32_t *pos, const float *topk_w,
                             int64_t T, int32_t k, int64_t d, uint16_t *out,
                             nvfp4moe_stream_t stream) {

@@ -792,7 +792,7 @@ int pair_grid() {
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     const bool nvf4 = a.kind == 0;
     const bool swiglu = a.epi == EPI_SWIGLU_AMAX;
-    if (swiglu && (!nvf4 || a.group_axis != NVFP4MOE_GROUP_M || (a.N / 2) % 128 != 0))
+    if (swiglu && (a.group_axis != NVFP4MOE_GROUP_M || (a.N / 2) % 128 != 0 || !a.amax))
         return cudaErrorInvalidValue;
     if (a.N % 256 != 0) return cudaErrorInvalidValue;
     // the per-group tile table packs the X-tile count of a group into 16 bits

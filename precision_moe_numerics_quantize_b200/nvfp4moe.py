@@ -57,6 +57,8 @@ _SIGS = {
                                             _P, _P, _P, _P, _P, _P]),
     "moe_expert_fwd": (C.c_int, [_P, _P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                  _P, _P, _P, _P, _P, _I64, _P]),
+    "moe_expert_fwd_mxfp8": (C.c_int, [_P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
+                                       _P, _P, _I64, _P]),
     "moe_combine": (C.c_int, [_P, _P, _P, _I64, _I32, _I64, _P, _P]),
     "moe_combine_rht": (C.c_int, [_P, _P, _P, _I, _U64, _P, _P, _I64, _I32, _I64, _P, _P]),
     "nvfp4_grouped_gemm": (C.c_int, [_P, _P, _P, _I32, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P,
@@ -205,6 +207,15 @@ def moe_expert_fwd(xq, xq_sc, x_ts, expert_off, E, d, f, w1, w1_sc, w1_ts, w2, w
         _ptr(xq), _ptr(xq_sc), _ptr(x_ts), _ptr(expert_off), E, d, f, _ptr(w1), _ptr(w1_sc),
         _ptr(w1_ts), _ptr(w2), _ptr(w2_sc), _ptr(w2_ts), _ptr(h), _ptr(hq), _ptr(hq_sc),
         _ptr(h_amax), _ptr(h_ts), _ptr(y), rows_alloc, _stream(stream)))
+
+
+def moe_expert_fwd_mxfp8(xq, xq_sc, expert_off, E, d, f, w1, w1_sc, w2, w2_sc, h, h_amax, hq,
+                         hq_sc, y, rows_alloc, stream=None):
+    """Expert FFN forward with MXFP8 operands (see include/nvfp4moe.h)."""
+    _check("moe_expert_fwd_mxfp8", lib().moe_expert_fwd_mxfp8(
+        _ptr(xq), _ptr(xq_sc), _ptr(expert_off), E, d, f, _ptr(w1), _ptr(w1_sc), _ptr(w2),
+        _ptr(w2_sc), _ptr(h), _ptr(h_amax), _ptr(hq), _ptr(hq_sc), _ptr(y), rows_alloc,
+        _stream(stream)))
 
 
 def moe_combine(y, pos, topk_w, out, stream=None):

@@ -217,3 +217,99 @@ def test_expert_fwd_small_layer(dev, lib, orc, router):
             assert np.all(ok[same]), e
         assert not gy[rows[tok[rows] < 0]].any()
     assert flips <= 1e-3 * total, (flips, total)
+
+
+def _mx_experts(orc, seed, tag, E, rows, cols):
+    cs, ss = [], []
+    for e in range(E):
+        W = _f32(synth.expert_weight_np(seed, tag, e, rows, cols))
+        c, s = orc.mxfp8_quantize(W, axis=0, rounding=0)
+        cs.append(c); ss.append(s)
+    return np.concatenate(cs), np.concatenate(ss)
+
+
+def _mx_f64(orc, codes, scales):
+    return orc.mxfp8_dequantize(codes, scales).astype(np.float64)
+
+
+@pytest.mark.parametrize("router", ["uniform", "zipf"])
+def test_expert_fwd_mxfp8_small_layer(dev, lib, orc, router):
+    """MXFP8 expert forward, 2048 tokens, d = 1024, f = 512, 32 experts, top-4.
+    h within one bf16 ulp plus the accumulator tolerance through SwiGLU; the
+    fused h_amax equals max|h|; every 32-block of hq whose h block agrees with
+    the oracle's has the oracle's codes and scale; y on rows whose hq agrees."""
+    sh = synth.SHAPES["small_moe"]
+    T, d, f, E, k = sh.T, sh.d, sh.f, sh.E, sh.k
+    logits = (synth.logits_uniform_np(2, T, E) if router == "uniform"
+              else synth.logits_zipf_np(2, T, E))
+    x = _f32(synth.rows_np(0, synth.TAG_X, 0, T, d, 1.0))
+    idx, _ = orc.route(logits, k)
+    off, pos, tok = orc.permute(idx, E)
+    xc_t, xs_t = orc.mxfp8_quantize(x, axis=0, rounding=0)
+    R = lib.max_rows(T, k, E)
+    xq = np.zeros((R, d), np.uint8)
+    xsc = np.zeros((R, d // 32), np.uint8)
+    real = np.where(tok >= 0)[0]
+    xq[real] = xc_t[tok[real]]
+    xsc[real] = xs_t[tok[real]]
+    w1c, w1s = _mx_experts(orc, 1, synth.TAG_W1, E, 2 * f, d)
+    w2c, w2s = _mx_experts(orc, 1, synth.TAG_W2, E, d, f)
+    h = torch.empty(R, f, dtype=torch.bfloat16, device=dev)
+    h_amax = torch.empty(E, device=dev)
+    hq = torch.empty(R, f, dtype=torch.uint8, device=dev)
+    hq_sc = torch.empty(R * f // 32, dtype=torch.uint8, device=dev)
+    y = torch.empty(R, d, dtype=torch.bfloat16, device=dev)
+    lib.moe_expert_fwd_mxfp8(dev_u8(xq, dev), dev_u8(rowmajor_to_mma(xsc), dev),
+                             torch.tensor(off, device=dev), E, d, f, dev_u8(w1c, dev),
+                             dev_u8(rowmajor_to_mma(w1s), dev), dev_u8(w2c, dev),
+                             dev_u8(rowmajor_to_mma(w2s), dev), h, h_amax, hq, hq_sc, y, R)
+    sync()
+    gh = _f32(host_bits(h)).astype(np.float64)
+    ghb = host_bits(h)
+    ghq = host_u8(hq)
+    ghs = mma_to_rowmajor(host_u8(hq_sc), R, f // 32)
+    gy = _f32(host_bits(y)).astype(np.float64)
+    gam = h_amax.cpu().numpy()
+    blocks = total_blocks = 0
+    for e in range(E):
+        rows = np.arange(off[e], off[e + 1])
+        rows_real = rows[tok[rows] >= 0]
+        if len(rows_real) == 0:
+            assert gam[e] == 0.0
+            continue
+        n = len(rows_real)
+        W1 = slice(e * 2 * f, (e + 1) * 2 * f)
+        W2 = slice(e * d, (e + 1) * d)
+        r = orc.expert_ffn_mxfp8(xq[rows_real], xsc[rows_real], w1c[W1], w1s[W1], w2c[W2],
+                                 w2s[W2])
+        A = _mx_f64(orc, xq[rows_real], xsc[rows_real])
+        B1 = _mx_f64(orc, w1c[W1], w1s[W1])
+        gu = orc.gemm_f64(A, B1)
+        mag = orc.gemm_f64(np.abs(A), np.abs(B1)) * 1e-5
+        g, u = gu[:, :f], gu[:, f:]
+        sig = 1.0 / (1.0 + np.exp(-g))
+        href = _f32(r["h"]).astype(np.float64)
+        tol = (_ulp(href) + np.abs(sig * (1 + g * (1 - sig)) * u) * mag[:, :f]
+               + np.abs(g * sig) * mag[:, f:] + 1e-30)
+        assert np.all(np.abs(gh[rows_real] - href) <= tol), e
+        assert gam[e] == np.abs(gh[rows]).max()
+        assert not gh[rows[tok[rows] < 0]].any()
+        # hq per 32-block: where the block of h is bit-identical, so are the
+        # block's codes and scale
+        hb_same = np.all((ghb[rows_real] == r["h"]).reshape(n, f // 32, 32), axis=2)
+        codes_same = np.all((ghq[rows_real] == r["hq"]).reshape(n, f // 32, 32), axis=2)
+        sc_same = ghs[rows_real] == r["hq_sc"]
+        assert np.all(codes_same[hb_same] & sc_same[hb_same]), e
+        blocks += int(hb_same.sum())
+        total_blocks += hb_same.size
+        # y on rows whose hq agrees
+        same = np.all(ghq[rows_real] == r["hq"], axis=1) & np.all(ghs[rows_real] == r["hq_sc"], axis=1)
+        H = _mx_f64(orc, r["hq"], r["hq_sc"])
+        B2 = _mx_f64(orc, w2c[W2], w2s[W2])
+        ymag = orc.gemm_f64(np.abs(H), np.abs(B2)) * 1e-5
+        yref = _f32(r["y"]).astype(np.float64)
+        ok = np.abs(gy[rows_real] - yref) <= _ulp(yref) * 2 + ymag + 1e-30
+        assert np.all(ok[same]), e
+        assert not gy[rows[tok[rows] < 0]].any()
+    # h itself agrees bit for bit in almost every block
+    assert blocks >= 0.99 * total_blocks, (blocks, total_blocks)
