@@ -37,10 +37,10 @@ if ROOT not in sys.path:
 
 METRIC = "NVFP4 expert-FFN fwd TFLOPS (% of B200 FP4 peak); quantizer HBM GB/s"
 # dram__bytes_read.sum + dram__bytes_write.sum of moe_expert_fwd's three
-# kernels (GEMM1 + SwiGLU 5.625 GB, requantize 0.953 GB, GEMM2 3.667 GB) per
+# kernels (GEMM1 + SwiGLU 5.627 GB, requantize 0.950 GB, GEMM2 3.676 GB) per
 # call of the full-size layer, from a 1-pass ncu capture of the current
 # kernels (summary under profiles/). Set back to None when they change.
-EXPERT_FWD_DRAM_BYTES = 10.245e9
+EXPERT_FWD_DRAM_BYTES = 10.252e9
 
 
 def load_peaks():

@@ -702,20 +702,45 @@ __global__ void __launch_bounds__(256) nvfp4_quant_grouped_kernel(
         for (int e = threadIdx.x; e < E; e += blockDim.x) ts[e] = nvfp4_ts(amax[e]);
     const int64_t rows = s_off[E];
     const int64_t G = cols / 64;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t r = i / G, g = i - r * G;
-        int lo = 0, hi = E;  // largest e with s_off[e] <= r
-        while (hi - lo > 1) {
-            int mid = (lo + hi) >> 1;
-            if (s_off[mid] <= r) lo = mid; else hi = mid;
+    // each CTA owns one contiguous range of 64-element groups, so the rows a
+    // thread meets only move forward and so does their expert
+    const int64_t n = rows * G;
+    const int64_t chunk = (n + gridDim.x - 1) / gridDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * chunk;
+    const int64_t i1 = i0 + chunk < n ? i0 + chunk : n;
+    int e = -1;
+    float S_enc = 1.0f;
+    for (int64_t i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+        const int64_t r = i / G, g = i - r * G;
+        const uint4 *pv = reinterpret_cast<const uint4 *>(x + r * cols + g * 64);
+        uint4 raw[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) raw[j] = __ldg(pv + j);
+        int e1 = e;
+        if (e1 < 0) {
+            int lo = 0, hi = E;  // largest e with s_off[e] <= r
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (s_off[mid] <= r) lo = mid; else hi = mid;
+            }
+            e1 = lo;
         }
-        const float S_enc = nvfp4_senc(amax[lo]);
-        uint4 c0, c1;
-        uint32_t scw = nvfp4_quant64(x + r * cols + g * 64, S_enc, c0, c1);
+        while (e1 + 1 < E && s_off[e1 + 1] <= r) ++e1;
+        if (e1 != e) {
+            e = e1;
+            S_enc = nvfp4_senc(amax[e]);
+        }
+        uint32_t scw = 0, w[8];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            float v[16];
+            unpack8(raw[2 * b], v);
+            unpack8(raw[2 * b + 1], v + 8);
+            scw |= nvfp4_block16(v, S_enc, w[2 * b], w[2 * b + 1]) << (8 * b);
+        }
         uint4 *co = reinterpret_cast<uint4 *>(codes + r * (cols / 2) + g * 32);
-        co[0] = c0;
-        co[1] = c1;
+        co[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        co[1] = make_uint4(w[4], w[5], w[6], w[7]);
         *reinterpret_cast<uint32_t *>(scales + mma_sf_offset(r, g * 4, cols / 16)) = scw;
     }
 }

@@ -30,7 +30,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["nvfp4_quantize", "mxfp8_quantize_sr", "rht32_quantize", "moe_route_permute",
-              "moe_expert_fwd", "moe_combine", "nvfp4_grouped_gemm", "mxfp8_grouped_gemm"]:
+              "moe_expert_fwd", "moe_expert_fwd_mxfp8", "moe_combine", "nvfp4_grouped_gemm",
+              "mxfp8_grouped_gemm"]:
         assert n in names
     assert set(names) == set(M.EXPORTED), set(names) ^ set(M.EXPORTED)
 
@@ -71,6 +72,16 @@ P = 1 << 20  # a fake, 16-byte aligned "device pointer"; validation fails before
                                    1 << 20, None), 2),                               # d % 64
     (lambda L: L.moe_expert_fwd(P, P, P, P, 4, 384, 256, P, P, P, P, P, P, P, P, P, P, P, P,
                                 128, None), 2),                                      # d % 256
+    (lambda L: L.moe_expert_fwd_mxfp8(P, P, P, 4, 384, 256, P, P, P, P, P, P, P, P, P, 128,
+                                      None), 2),                                     # d % 256
+    (lambda L: L.moe_expert_fwd_mxfp8(P, P, P, 4, 256, 256, P, P, P, P, P, P, P, P, P, 100,
+                                      None), 2),                                     # rows % 128
+    (lambda L: L.moe_expert_fwd_mxfp8(P, P, P, 0, 256, 256, P, P, P, P, P, P, P, P, P, 128,
+                                      None), 1),                                     # E
+    (lambda L: L.moe_expert_fwd_mxfp8(P, P, P, 4, 256, 256, P, P, None, P, P, P, P, P, P, 128,
+                                      None), 1),                                     # null w2
+    (lambda L: L.moe_expert_fwd_mxfp8(P, P, P, 4, 256, 256, P, P, P, P, P + 2, P, P, P, P, 128,
+                                      None), 3),                                     # align h
     (lambda L: L.moe_combine(P, P, P, 4, 2, 12, P, None), 2),                        # d % 8
     (lambda L: L.nvfp4_grouped_gemm(P, P, P, 2, P, P, P, P, 1, 128, 256, 256, P, 0, None), 1),
     (lambda L: L.nvfp4_grouped_gemm(P, P, P, 0, P, P, P, P, 1, 128, 256, 128, P, 0, None), 2),
