@@ -765,6 +765,29 @@ ORACLE_API void oracle_expert_ffn_mxfp8(const uint8_t *xq, const uint8_t *xq_sc,
 }
 
 /*
+ * READING ([P1] "训练数值格式分工清单": the backward pass of the expert layers
+ * runs in MXFP8): the SwiGLU step of the backward pass. For h = silu(g) * u
+ * with silu(g) = g * s(g), s(g) = 1 / (1 + exp(-g)):
+ *   dg = dh * u * s(g) * (1 + g * (1 - s(g)))
+ *   du = dh * silu(g)
+ * gu_bits [rows x 2f] holds g in columns 0..f-1 and u in f..2f-1 (the layout
+ * GEMM1 writes), dh_bits [rows x f]; dgu_bits [rows x 2f] gets dg | du in the
+ * same layout, each computed in fp64 and rounded once to bf16.
+ */
+ORACLE_API void oracle_swiglu_bwd(const uint16_t *gu_bits, const uint16_t *dh_bits, int64_t rows,
+                                  int64_t f, uint16_t *dgu_bits) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < f; ++c) {
+            const double g = oracle_bf16_to_f32(gu_bits[r * 2 * f + c]);
+            const double u = oracle_bf16_to_f32(gu_bits[r * 2 * f + f + c]);
+            const double dh = oracle_bf16_to_f32(dh_bits[r * f + c]);
+            const double sg = 1.0 / (1.0 + exp(-g));
+            dgu_bits[r * 2 * f + c] = oracle_bf16_from_f64(dh * u * sg * (1.0 + g * (1.0 - sg)));
+            dgu_bits[r * 2 * f + f + c] = oracle_bf16_from_f64(dh * g * sg);
+        }
+}
+
+/*
  * READING ([P2] "Key Takeaways": the combine step): out[t] = sum over slots j
  * of w[t, j] * y[pos[t, j]] in fp64, rounded once to bf16. y rows are bf16.
  */

@@ -16,7 +16,7 @@ __all__ = [
     "nvfp4_to_f64", "philox4x32_10", "philox_word", "mxfp8_quantize", "mxfp8_dequantize",
     "rht_signs", "rht32_forward_f32", "rht32_inverse_f32", "rht32_f64", "rht32_quantize",
     "rht32_dequantize", "route", "permute", "gemm_f64", "swiglu", "expert_ffn", "combine",
-    "combine_f32", "combine_rht", "mxfp8_rpad", "expert_ffn_mxfp8",
+    "combine_f32", "combine_rht", "mxfp8_rpad", "expert_ffn_mxfp8", "swiglu_bwd",
 ]
 
 _lib = None
@@ -68,6 +68,7 @@ def _declare(L):
                                      _P, C.c_float, _P, _I64, _P, _P, _P, _P, _P]),
         "oracle_expert_ffn_mxfp8": (None, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _I64,
                                            _P, _P, _P, _P]),
+        "oracle_swiglu_bwd": (None, [_P, _P, _I64, _I64, _P]),
         "oracle_combine": (None, [_P, _P, _P, _I64, _I32, _I64, _P]),
         "oracle_combine_f32": (None, [_P, _P, _P, _I64, _I32, _I64, _P]),
         "oracle_combine_rht": (None, [_P, _P, C.c_float, C.c_int, _U64, _P, _P, _I64, _I32,
@@ -364,6 +365,17 @@ def expert_ffn_mxfp8(xq, xq_sc, w1, w1_sc, w2, w2_sc, rows_out=None):
                                   _p(w2_sc), _p(ro), 0 if ro is None else len(ro), _p(h), _p(hq),
                                   _p(hq_sc), _p(y))
     return {"h": h, "hq": hq, "hq_sc": hq_sc, "y": y}
+
+
+def swiglu_bwd(gu_bits, dh_bits):
+    """SwiGLU backward: gu bf16 bits [rows, 2f] (g | u), dh [rows, f] -> dg | du bf16 bits
+    [rows, 2f], fp64 arithmetic rounded once."""
+    gu_bits = _c(gu_bits, np.uint16)
+    dh_bits = _c(dh_bits, np.uint16)
+    rows, f = dh_bits.shape
+    out = np.zeros((rows, 2 * f), np.uint16)
+    lib().oracle_swiglu_bwd(_p(gu_bits), _p(dh_bits), rows, f, _p(out))
+    return out
 
 
 def combine(y_bits, pos, w):

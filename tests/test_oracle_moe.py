@@ -194,3 +194,24 @@ def test_combine_one_hot(orc):
         for j in range(k):
             assert out[t, (t + j) % d] == (1.0 + j) * 2.0 ** -j
     assert np.count_nonzero(out) == T * k
+
+
+def test_swiglu_bwd_matches_autograd(orc):
+    """The SwiGLU backward against torch autograd of silu(g) * u in fp64, both
+    rounded once to bf16 by torch; inputs include large |g| where s(g)
+    saturates, and dh = 0."""
+    rows, f = 64, 96
+    gu_bits = synth.rows_np(4, synth.TAG_ACT, 0, rows, 2 * f, 2.0)
+    gu_bits[0, :8] = synth.f32_to_bf16_bits(np.array([-100, -30, -8, 0, 8, 30, 100, 1e-3],
+                                                     np.float32))
+    dh_bits = synth.rows_np(5, synth.TAG_ACT, 0, rows, f, 0.5)
+    dh_bits[1, :] = 0
+    got = orc.swiglu_bwd(gu_bits, dh_bits)
+    gu = torch.from_numpy(synth.bf16_bits_to_f32(gu_bits).astype(np.float64))
+    g = gu[:, :f].clone().requires_grad_(True)
+    u = gu[:, f:].clone().requires_grad_(True)
+    dh = torch.from_numpy(synth.bf16_bits_to_f32(dh_bits).astype(np.float64))
+    (torch.nn.functional.silu(g) * u).backward(dh)
+    ref = torch.cat([g.grad, u.grad], dim=1).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+    assert not synth.bf16_bits_to_f32(got[1]).any()
