@@ -395,6 +395,14 @@ def companions(M, synth, torch, dev, L, peaks, reps=10):
                                "note": "fp32 dW [E x d x f] written"}
     del dW, dy, act, dyc0, dys0, dyc1, dys1, ac1, as1, w2c, w2s
     torch.cuda.empty_cache()
+    # SwiGLU backward on the routed rows: g | u [Rp x 2f] and dh [Rp x f] in,
+    # dg | du [Rp x 2f] out (6 bytes read, 4 written per column pair)
+    gu_t = synth.rows_torch(9, synth.TAG_ACT, 0, Rp, 2 * f, 2.0, dev)
+    dh_t = synth.rows_torch(10, synth.TAG_ACT, 0, Rp, f, 0.5, dev)
+    dgu_t = torch.empty_like(gu_t)
+    gbs("swiglu_bwd", lambda: M.swiglu_bwd(gu_t, dh_t, dgu_t), Rp * f, 10)
+    del gu_t, dh_t, dgu_t
+    torch.cuda.empty_cache()
     # The expert FFN forward in MXFP8 (the layers that stay in MXFP8): the same
     # routed rows, x / W1 / W2 quantized along rows with round-to-nearest-even
     R = L["R"]

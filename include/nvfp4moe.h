@@ -300,6 +300,21 @@ nvfp4moe_status moe_expert_fwd_mxfp8(const uint8_t *xq, const uint8_t *xq_sc,
                                      nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * SwiGLU backward (news.t0001.com '训练数值格式分工清单': the backward pass of
+ * the expert layers runs in MXFP8; this is its elementwise SwiGLU step, whose
+ * output is quantized with mxfp8_quantize_sr for the GEMM1 dgrad and wgrad).
+ * gu bf16 [rows x 2f]: g in columns 0..f-1, u in f..2f-1 (the layout GEMM1
+ * writes with out = X . W1^T, W1 = [gate; up]). dh bf16 [rows x f], the
+ * gradient of h = silu(g) * u. Writes dgu bf16 [rows x 2f] = dg | du:
+ *   dg = dh * u * s(g) * (1 + g * (1 - s(g))),  du = dh * g * s(g),
+ *   s(g) = 1 / (1 + exp(-g)), fp32 arithmetic, bf16 round-to-nearest-even.
+ * f % 8 == 0; pointers 16-byte aligned; dgu must not overlap the inputs.
+ * rows = 0 is a no-op. Errors: NVFP4MOE_ERR_INVALID_ARG, _SHAPE, _ALIGN
+ * before any launch; NVFP4MOE_ERR_CUDA for a failed launch. */
+nvfp4moe_status swiglu_bwd(const uint16_t *gu, const uint16_t *dh, int64_t rows, int64_t f,
+                           uint16_t *dgu, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Weighted top-k combine (aicoder.com 'Key Takeaways': the combine step).
  * out[t] = bf16( sum_{j=0..k-1} topk_w[t,j] * y[pos[t,j]] ), fp32 accumulation
  * in slot order with fused multiply-adds; a gather, no atomics.

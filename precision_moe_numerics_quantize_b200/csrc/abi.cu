@@ -401,6 +401,17 @@ nvfp4moe_status moe_expert_fwd_mxfp8(const uint8_t *xq, const uint8_t *xq_sc,
     return after_launch(cudaSuccess, "moe_expert_fwd_mxfp8");
 }
 
+nvfp4moe_status swiglu_bwd(const uint16_t *gu, const uint16_t *dh, int64_t rows, int64_t f,
+                           uint16_t *dgu, nvfp4moe_stream_t stream) {
+    NEED(rows >= 0 && f > 0, NVFP4MOE_ERR_INVALID_ARG, "swiglu_bwd: sizes");
+    NEED(f % 8 == 0, NVFP4MOE_ERR_SHAPE, "swiglu_bwd: f %% 8 == 0 required");
+    if (rows > 0) {
+        NEED_PTR(gu); NEED_PTR(dh); NEED_PTR(dgu);
+        NEED(dgu != gu && dgu != dh, NVFP4MOE_ERR_INVALID_ARG, "swiglu_bwd: dgu aliases an input");
+    }
+    return after_launch(launch_swiglu_bwd(gu, dh, rows, f, dgu, (cudaStream_t)stream), "swiglu_bwd");
+}
+
 nvfp4moe_status moe_combine(const uint16_t *y, const int32_t *pos, const float *topk_w,
                             int64_t T, int32_t k, int64_t d, uint16_t *out,
                             nvfp4moe_stream_t stream) {

@@ -756,6 +756,54 @@ cudaError_t launch_nvfp4_quant_grouped(const uint16_t *x, int64_t rows_alloc, in
 }
 
 // ---------------------------------------------------------------------------
+// SwiGLU backward (the backward pass of the expert layers, news.t0001.com
+// "训练数值格式分工清单"): from the saved g | u and dh,
+//   dg = dh * u * s(g) * (1 + g * (1 - s(g))),  du = dh * g * s(g),
+// s(g) = 1 / (1 + exp(-g)), in fp32 with IEEE division, rounded to bf16.
+// One thread per 8 columns of a row: three 16-byte loads, two 16-byte stores.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) swiglu_bwd_kernel(const uint16_t *__restrict__ gu,
+                                                         const uint16_t *__restrict__ dh,
+                                                         int64_t rows, int64_t f,
+                                                         uint16_t *__restrict__ dgu) {
+    const int64_t G = f / 8;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * G;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / G, c = (i - r * G) * 8;
+        const uint16_t *row = gu + r * 2 * f;
+        const uint4 qg = __ldg(reinterpret_cast<const uint4 *>(row + c));
+        const uint4 qu = __ldg(reinterpret_cast<const uint4 *>(row + f + c));
+        const uint4 qd = __ldg(reinterpret_cast<const uint4 *>(dh + r * f + c));
+        float g[8], u[8], d[8];
+        unpack_bf16x8(qg, g);
+        unpack_bf16x8(qu, u);
+        unpack_bf16x8(qd, d);
+        float dg[8], du[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float sg = 1.0f / (1.0f + expf(-g[j]));
+            const float ds = sg * (1.0f + g[j] * (1.0f - sg));  // d silu / d g
+            dg[j] = d[j] * u[j] * ds;
+            du[j] = d[j] * (g[j] * sg);
+        }
+        uint16_t *orow = dgu + r * 2 * f;
+        *reinterpret_cast<uint4 *>(orow + c) =
+            make_uint4(bf16x2_rn(dg[0], dg[1]), bf16x2_rn(dg[2], dg[3]), bf16x2_rn(dg[4], dg[5]),
+                       bf16x2_rn(dg[6], dg[7]));
+        *reinterpret_cast<uint4 *>(orow + f + c) =
+            make_uint4(bf16x2_rn(du[0], du[1]), bf16x2_rn(du[2], du[3]), bf16x2_rn(du[4], du[5]),
+                       bf16x2_rn(du[6], du[7]));
+    }
+}
+
+cudaError_t launch_swiglu_bwd(const uint16_t *gu, const uint16_t *dh, int64_t rows, int64_t f,
+                              uint16_t *dgu, cudaStream_t s) {
+    if (rows * f == 0) return cudaSuccess;
+    swiglu_bwd_kernel<<<grid_for(rows * (f / 8)), 256, 0, s>>>(gu, dh, rows, f, dgu);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Self-test of the hardware conversions the quantizers use: every finite fp32
 // input, hardware result against the library's software encoders.
 // which 0: cvt.rn.satfinite.e2m1x2.f32; which 1: cvt.rn.satfinite.e4m3x2.f32.

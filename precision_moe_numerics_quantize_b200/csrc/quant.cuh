@@ -32,6 +32,8 @@ cudaError_t launch_nvfp4_quant_grouped(const uint16_t *x, int64_t rows_alloc, in
                                        uint8_t *codes, uint8_t *scales, float *ts,
                                        cudaStream_t s);
 
+cudaError_t launch_swiglu_bwd(const uint16_t *gu, const uint16_t *dh, int64_t rows, int64_t f,
+                              uint16_t *dgu, cudaStream_t s);
 cudaError_t launch_selftest(int which, unsigned long long *mismatches, cudaStream_t s);
 
 // routing / permutation / combine (route.cu)

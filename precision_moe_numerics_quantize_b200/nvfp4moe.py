@@ -59,6 +59,7 @@ _SIGS = {
                                  _P, _P, _P, _P, _P, _I64, _P]),
     "moe_expert_fwd_mxfp8": (C.c_int, [_P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _I64, _P]),
+    "swiglu_bwd": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "moe_combine": (C.c_int, [_P, _P, _P, _I64, _I32, _I64, _P, _P]),
     "moe_combine_rht": (C.c_int, [_P, _P, _P, _I, _U64, _P, _P, _I64, _I32, _I64, _P, _P]),
     "nvfp4_grouped_gemm": (C.c_int, [_P, _P, _P, _I32, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P,
@@ -216,6 +217,12 @@ def moe_expert_fwd_mxfp8(xq, xq_sc, expert_off, E, d, f, w1, w1_sc, w2, w2_sc, h
         _ptr(xq), _ptr(xq_sc), _ptr(expert_off), E, d, f, _ptr(w1), _ptr(w1_sc), _ptr(w2),
         _ptr(w2_sc), _ptr(h), _ptr(h_amax), _ptr(hq), _ptr(hq_sc), _ptr(y), rows_alloc,
         _stream(stream)))
+
+
+def swiglu_bwd(gu, dh, dgu, stream=None):
+    """SwiGLU backward: gu [rows, 2f] (g | u), dh [rows, f] -> dgu [rows, 2f] (dg | du), bf16."""
+    rows, f = dh.shape
+    _check("swiglu_bwd", lib().swiglu_bwd(_ptr(gu), _ptr(dh), rows, f, _ptr(dgu), _stream(stream)))
 
 
 def moe_combine(y, pos, topk_w, out, stream=None):
