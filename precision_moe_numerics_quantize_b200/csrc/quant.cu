@@ -234,96 +234,83 @@ __global__ void __launch_bounds__(256) mxfp8_rows_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// MXFP8 along columns, transposed output. A CTA stages a 128-row x 256-column
-// tile in shared memory with coalesced 16-byte loads. Thread t owns the four
-// adjacent columns 4 * (t % 64) .. +3 of the 32-row block t / 64: those four
+// MXFP8 along columns, transposed output. A warp owns a 32-row x 32-column
+// patch: lane = 8 rq + cq holds rows 8 rq .. 8 rq + 7 of the patch's 32-row
+// block and the four adjacent columns 4 cq .. 4 cq + 3. It reads them straight
+// from global memory (each row a 64-byte run per row quarter), the block amax
+// of a column joins its four row quarters with two shuffles, and the four
 // elements of a row are consecutive in the source, so one Philox call per row
-// gives all four of them their random words.
+// gives all four their random words. No shared memory: occupancy is set by
+// registers alone.
 // ---------------------------------------------------------------------------
-constexpr int MXC_TR = 128, MXC_TC = 256, MXC_LD = MXC_TC + 8;
-constexpr size_t MXC_SMEM = sizeof(uint16_t) * MXC_TR * MXC_LD;
-
 template <bool SR>
-__global__ void __launch_bounds__(256) mxfp8_cols_kernel(
+__global__ void __launch_bounds__(256, 3) mxfp8_cols_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
     uint64_t offset, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int layout) {
-    extern __shared__ __align__(16) uint16_t tile[];
-    const int64_t row_tiles = (rows + MXC_TR - 1) / MXC_TR;
-    const int64_t col_tiles = (cols + MXC_TC - 1) / MXC_TC;
-    const int64_t G = rows / 32;  // scales per output row
-    for (int64_t t = blockIdx.x; t < row_tiles * col_tiles; t += gridDim.x) {
-        const int64_t r0 = (t / col_tiles) * MXC_TR, c0 = (t % col_tiles) * MXC_TC;
-        const int nr = (int)(rows - r0 < MXC_TR ? rows - r0 : MXC_TR);
-        const int nc = (int)(cols - c0 < MXC_TC ? cols - c0 : MXC_TC);
-        __syncthreads();
-        for (int v = threadIdx.x; v < MXC_TR * (MXC_TC / 8); v += 256) {
-            const int rr = v / (MXC_TC / 8), cc = (v % (MXC_TC / 8)) * 8;
-            uint4 q = make_uint4(0, 0, 0, 0);
-            if (rr < nr && cc < nc) q = __ldg(reinterpret_cast<const uint4 *>(x + (r0 + rr) * ld + c0 + cc));
-            *reinterpret_cast<uint4 *>(&tile[rr * MXC_LD + cc]) = q;
-        }
-        __syncthreads();
-        const int cl = (threadIdx.x & 63) * 4, rb = threadIdx.x >> 6;
-        if (rb * 32 >= nr || cl >= nc) continue;
-        const uint16_t *tp = tile + (rb * 32) * MXC_LD + cl;
+    const int lane = threadIdx.x & 31, rq = lane >> 3, cq = lane & 7;
+    const int64_t G = rows / 32;          // scales per output row
+    const int64_t CP = cols / 32;         // column patches
+    const int64_t items = G * CP;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t it = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+         it += warps) {
+        const int64_t b = it / CP, cp = it - b * CP;
+        const int64_t r0 = b * 32 + rq * 8, c = cp * 32 + cq * 4;
+        uint2 q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __ldg(reinterpret_cast<const uint2 *>(x + (r0 + i) * ld + c));
         float am0 = 0.0f, am1 = 0.0f, am2 = 0.0f, am3 = 0.0f;
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-            const uint2 q = *reinterpret_cast<const uint2 *>(tp + i * MXC_LD);
-            am0 = fmaxf(am0, fabsf(bf16_lo(q.x)));
-            am1 = fmaxf(am1, fabsf(bf16_hi(q.x)));
-            am2 = fmaxf(am2, fabsf(bf16_lo(q.y)));
-            am3 = fmaxf(am3, fabsf(bf16_hi(q.y)));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            am0 = fmaxf(am0, fabsf(bf16_lo(q[i].x)));
+            am1 = fmaxf(am1, fabsf(bf16_hi(q[i].x)));
+            am2 = fmaxf(am2, fabsf(bf16_lo(q[i].y)));
+            am3 = fmaxf(am3, fabsf(bf16_hi(q[i].y)));
+        }
+#pragma unroll
+        for (int m = 8; m <= 16; m <<= 1) {
+            am0 = fmaxf(am0, __shfl_xor_sync(0xFFFFFFFFu, am0, m));
+            am1 = fmaxf(am1, __shfl_xor_sync(0xFFFFFFFFu, am1, m));
+            am2 = fmaxf(am2, __shfl_xor_sync(0xFFFFFFFFu, am2, m));
+            am3 = fmaxf(am3, __shfl_xor_sync(0xFFFFFFFFu, am3, m));
         }
         const int k0 = mx_scale_exp(am0), k1 = mx_scale_exp(am1), k2 = mx_scale_exp(am2),
                   k3 = mx_scale_exp(am3);
-        const int64_t rbase = r0 + rb * 32, c = c0 + cl;
-        uint32_t w0[8], w1[8], w2[8], w3[8];
+        // code bytes of rows r0 .. r0 + 7, per column: [column][row half]
+        uint32_t w0[2] = {0u, 0u}, w1[2] = {0u, 0u}, w2[2] = {0u, 0u}, w3[2] = {0u, 0u};
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+        for (int i = 0; i < 8; ++i) {
+            float v0 = scale_pow2(bf16_lo(q[i].x), k0), v1 = scale_pow2(bf16_hi(q[i].x), k1);
+            float v2 = scale_pow2(bf16_lo(q[i].y), k2), v3 = scale_pow2(bf16_hi(q[i].y), k3);
+            if (SR) {
+                // elements (r0 + i, c .. c + 3): row-major index multiple of 4
+                const u32x4 r4 = philox_block(seed, offset, (uint64_t)((r0 + i) * cols + c) >> 2);
+                v0 = e4m3_sr_value(v0, r4.x);
+                v1 = e4m3_sr_value(v1, r4.y);
+                v2 = e4m3_sr_value(v2, r4.z);
+                v3 = e4m3_sr_value(v3, r4.w);
+            }
+            const uint32_t p01 = e4m3x2_hw(v0, v1), p23 = e4m3x2_hw(v2, v3);
+            const int h = i >> 2, sh = 8 * (i & 3);
+            w0[h] |= (p01 & 0xFFu) << sh;
+            w1[h] |= (p01 >> 8) << sh;
+            w2[h] |= (p23 & 0xFFu) << sh;
+            w3[h] |= (p23 >> 8) << sh;
+        }
+        *reinterpret_cast<uint2 *>(codes + (c + 0) * rows + r0) = make_uint2(w0[0], w0[1]);
+        *reinterpret_cast<uint2 *>(codes + (c + 1) * rows + r0) = make_uint2(w1[0], w1[1]);
+        *reinterpret_cast<uint2 *>(codes + (c + 2) * rows + r0) = make_uint2(w2[0], w2[1]);
+        *reinterpret_cast<uint2 *>(codes + (c + 3) * rows + r0) = make_uint2(w3[0], w3[1]);
+        if (rq == 0) {
+            const int ks[4] = {k0, k1, k2, k3};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int i = 4 * q + j;
-                const uint2 pr = *reinterpret_cast<const uint2 *>(tp + i * MXC_LD);
-                const float v0 = scale_pow2(bf16_lo(pr.x), k0), v1 = scale_pow2(bf16_hi(pr.x), k1);
-                const float v2 = scale_pow2(bf16_lo(pr.y), k2), v3 = scale_pow2(bf16_hi(pr.y), k3);
-                uint32_t e0, e1, e2, e3;
-                float w0v = v0, w1v = v1, w2v = v2, w3v = v3;
-                if (SR) {
-                    // elements (rbase + i, c .. c + 3): row-major index multiple of 4
-                    const u32x4 r4 = philox_block(seed, offset, (uint64_t)((rbase + i) * cols + c) >> 2);
-                    w0v = e4m3_sr_value(v0, r4.x);
-                    w1v = e4m3_sr_value(v1, r4.y);
-                    w2v = e4m3_sr_value(v2, r4.z);
-                    w3v = e4m3_sr_value(v3, r4.w);
-                }
-                const uint32_t p01 = e4m3x2_hw(w0v, w1v), p23 = e4m3x2_hw(w2v, w3v);
-                e0 = p01 & 0xFFu; e1 = p01 >> 8; e2 = p23 & 0xFFu; e3 = p23 >> 8;
-                a0 |= e0 << (8 * j);
-                a1 |= e1 << (8 * j);
-                a2 |= e2 << (8 * j);
-                a3 |= e3 << (8 * j);
+                const uint8_t e8 = (uint8_t)(ks[j] + 127);
+                if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
+                    scales[(c + j) * G + b] = e8;
+                else
+                    scales[mma_sf_offset(c + j, b, G)] = e8;
             }
-            w0[q] = a0; w1[q] = a1; w2[q] = a2; w3[q] = a3;
-        }
-        uint4 *o0 = reinterpret_cast<uint4 *>(codes + (c + 0) * rows + rbase);
-        uint4 *o1 = reinterpret_cast<uint4 *>(codes + (c + 1) * rows + rbase);
-        uint4 *o2 = reinterpret_cast<uint4 *>(codes + (c + 2) * rows + rbase);
-        uint4 *o3 = reinterpret_cast<uint4 *>(codes + (c + 3) * rows + rbase);
-        o0[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]); o0[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
-        o1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]); o1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
-        o2[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]); o2[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
-        o3[0] = make_uint4(w3[0], w3[1], w3[2], w3[3]); o3[1] = make_uint4(w3[4], w3[5], w3[6], w3[7]);
-        const int64_t b = rbase / 32;
-        const int ks[4] = {k0, k1, k2, k3};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint8_t e8 = (uint8_t)(ks[j] + 127);
-            if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
-                scales[(c + j) * G + b] = e8;
-            else
-                scales[mma_sf_offset(c + j, b, G)] = e8;
         }
     }
 }
@@ -619,25 +606,14 @@ cudaError_t launch_mxfp8_quantize(const uint16_t *x, int64_t rows, int64_t cols,
             mxfp8_rows_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes,
                                                        scales, layout);
     } else {
-        static bool attr = false;
-        if (!attr) {
-            cudaError_t e = cudaFuncSetAttribute(mxfp8_cols_kernel<true>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)MXC_SMEM);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(mxfp8_cols_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MXC_SMEM);
-            if (e != cudaSuccess) return e;
-            attr = true;
-        }
-        int64_t tiles = ((rows + MXC_TR - 1) / MXC_TR) * ((cols + MXC_TC - 1) / MXC_TC);
-        int g = (int)(tiles < 148 * 3 ? tiles : 148 * 3);
+        // one warp per 32 x 32 patch, 8 warps per CTA
+        const int g = grid_for((rows / 32) * (cols / 32), 8);
         if (sr)
-            mxfp8_cols_kernel<true><<<g, 256, MXC_SMEM, s>>>(x, rows, cols, ld, seed, offset, codes,
-                                                             scales, layout);
+            mxfp8_cols_kernel<true><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes, scales,
+                                                      layout);
         else
-            mxfp8_cols_kernel<false><<<g, 256, MXC_SMEM, s>>>(x, rows, cols, ld, seed, offset,
-                                                              codes, scales, layout);
+            mxfp8_cols_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes,
+                                                       scales, layout);
     }
     return cudaGetLastError();
 }
