@@ -207,7 +207,7 @@ NV_DEV uint32_t mx_block32(const float (&v)[32], uint64_t seed, uint64_t offset,
 }
 
 template <bool SR>
-__global__ void __launch_bounds__(256) mxfp8_rows_kernel(
+__global__ void __launch_bounds__(256, 4) mxfp8_rows_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
     uint64_t offset, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int layout) {
     const uint32_t G = (uint32_t)(cols / 32);  // blocks per row
