@@ -84,7 +84,7 @@ typedef enum {
     NVFP4MOE_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query says */
     NVFP4MOE_ERR_CUDA = 5,        /* a CUDA call failed; see nvfp4moe_last_error() */
     NVFP4MOE_ERR_TIMEOUT = 6,     /* a bounded device wait ran out (nvfp4moe_device_error) */
-    NVFP4MOE_ERR_UNSUPPORTED = 7  /* valid request this build does not implement */
+    NVFP4MOE_ERR_UNSUPPORTED = 7  /* valid request this library version does not implement */
 } nvfp4moe_status;
 
 enum { NVFP4MOE_LAYOUT_ROWMAJOR = 0, NVFP4MOE_LAYOUT_MMA = 1 };
