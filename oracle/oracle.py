@@ -17,6 +17,7 @@ __all__ = [
     "rht_signs", "rht32_forward_f32", "rht32_inverse_f32", "rht32_f64", "rht32_quantize",
     "rht32_dequantize", "route", "permute", "gemm_f64", "swiglu", "expert_ffn", "combine",
     "combine_f32", "combine_rht", "mxfp8_rpad", "expert_ffn_mxfp8", "swiglu_bwd",
+    "expert_bwd_gemm1",
 ]
 
 _lib = None
@@ -376,6 +377,31 @@ def swiglu_bwd(gu_bits, dh_bits):
     out = np.zeros((rows, 2 * f), np.uint16)
     lib().oracle_swiglu_bwd(_p(gu_bits), _p(dh_bits), rows, f, _p(out))
     return out
+
+
+def expert_bwd_gemm1(dgu_bits, x_bits, w1_bits, seed=0, offset=0):
+    """GEMM1's backward for one expert in MXFP8 ([P1] "训练数值格式分工清单" and [P2]
+    "Architecture highlights": the backward pass runs in MXFP8, the gradients
+    with stochastic rounding). With dgu [n, 2f] the gradient of g | u (bf16
+    bits), x [n, d] the expert's input rows and W1 [2f, d] (bf16 bits):
+      dX  = dq(SR(dgu) along 2f) . dq(RNE(W1) along 2f)    -> bf16 [n, d]
+      dW1 = dq(SR(dgu) along n)^T . dq(RNE(x) along n)     -> fp32 [2f, d]
+    The row-wise stochastic rounding draws from (seed, offset), the
+    column-wise one from (seed, offset + 1); blocks along n are padded to 32
+    rows with zeros. Products are summed in fp64 and rounded once."""
+    dgu = bf16_to_f32(_c(dgu_bits, np.uint16))
+    x = bf16_to_f32(_c(x_bits, np.uint16))
+    w1 = bf16_to_f32(_c(w1_bits, np.uint16))
+    n, f2 = dgu.shape
+    # dgrad: contraction over 2f
+    gc, gs = mxfp8_quantize(dgu, axis=0, seed=seed, offset=offset, rounding=1)
+    wc, ws = mxfp8_quantize(w1, axis=1, rounding=0)            # [d, 2f]
+    dx = gemm_f64(mxfp8_dequantize(gc, gs), mxfp8_dequantize(wc, ws))
+    # wgrad: contraction over the expert's rows
+    tc, ts = mxfp8_quantize(dgu, axis=1, seed=seed, offset=offset + 1, rounding=1)  # [2f, npad]
+    xc, xs = mxfp8_quantize(x, axis=1, rounding=0)             # [d, npad]
+    dw = gemm_f64(mxfp8_dequantize(tc, ts), mxfp8_dequantize(xc, xs))
+    return {"dx": bf16_from_f64(dx), "dw1": dw.astype(np.float32)}
 
 
 def combine(y_bits, pos, w):
