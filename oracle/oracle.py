@@ -379,29 +379,46 @@ def swiglu_bwd(gu_bits, dh_bits):
     return out
 
 
-def expert_bwd_gemm1(dgu_bits, x_bits, w1_bits, seed=0, offset=0):
-    """GEMM1's backward for one expert in MXFP8 ([P1] "训练数值格式分工清单" and [P2]
-    "Architecture highlights": the backward pass runs in MXFP8, the gradients
-    with stochastic rounding). With dgu [n, 2f] the gradient of g | u (bf16
-    bits), x [n, d] the expert's input rows and W1 [2f, d] (bf16 bits):
-      dX  = dq(SR(dgu) along 2f) . dq(RNE(W1) along 2f)    -> bf16 [n, d]
-      dW1 = dq(SR(dgu) along n)^T . dq(RNE(x) along n)     -> fp32 [2f, d]
-    The row-wise stochastic rounding draws from (seed, offset), the
-    column-wise one from (seed, offset + 1); blocks along n are padded to 32
-    rows with zeros. Products are summed in fp64 and rounded once."""
+def expert_bwd_gemm1(dgu_bits, x_bits, w1_bits, expert_off=None, seed=0, offset=0):
+    """GEMM1's backward in MXFP8 for a grouped layer ([P1] "训练数值格式分工清单" and
+    [P2] "Architecture highlights": the backward pass runs in MXFP8, the
+    gradients with stochastic rounding). dgu [R, 2f] is the gradient of g | u
+    and x [R, d] the experts' input rows (bf16 bits), expert e owning rows
+    expert_off[e] .. expert_off[e+1] (None: one expert, all rows); W1 [E, 2f, d].
+      dX_e  = dq(SR(dgu) along 2f)_e . dq(RNE(W1_e) along 2f)    -> bf16 [R, d]
+      dW1_e = dq(SR(dgu) along rows)_e^T . dq(RNE(x) along rows)_e -> fp32 [E, 2f, d]
+    The stochastic draws follow each element's row-major index in the whole
+    [R, 2f] tensor: row-wise from (seed, offset), column-wise from
+    (seed, offset + 1). Column blocks run within each expert's rows, padded to
+    32 with zero rows. Products are summed in fp64 and rounded once."""
     dgu = bf16_to_f32(_c(dgu_bits, np.uint16))
     x = bf16_to_f32(_c(x_bits, np.uint16))
     w1 = bf16_to_f32(_c(w1_bits, np.uint16))
-    n, f2 = dgu.shape
+    if w1.ndim == 2:
+        w1 = w1[None]
+    R, f2 = dgu.shape
+    off = np.array([0, R], np.int32) if expert_off is None else _c(expert_off, np.int32)
+    E = len(off) - 1
     # dgrad: contraction over 2f
     gc, gs = mxfp8_quantize(dgu, axis=0, seed=seed, offset=offset, rounding=1)
-    wc, ws = mxfp8_quantize(w1, axis=1, rounding=0)            # [d, 2f]
-    dx = gemm_f64(mxfp8_dequantize(gc, gs), mxfp8_dequantize(wc, ws))
-    # wgrad: contraction over the expert's rows
-    tc, ts = mxfp8_quantize(dgu, axis=1, seed=seed, offset=offset + 1, rounding=1)  # [2f, npad]
-    xc, xs = mxfp8_quantize(x, axis=1, rounding=0)             # [d, npad]
-    dw = gemm_f64(mxfp8_dequantize(tc, ts), mxfp8_dequantize(xc, xs))
-    return {"dx": bf16_from_f64(dx), "dw1": dw.astype(np.float32)}
+    G = mxfp8_dequantize(gc, gs)
+    # wgrad: contraction over each expert's rows; the padded segments follow
+    # one another in the transposed outputs
+    tc, ts = mxfp8_quantize(dgu, axis=1, seg_off=off, seed=seed, offset=offset + 1, rounding=1)
+    xc, xs = mxfp8_quantize(x, axis=1, seg_off=off, rounding=0)
+    Tq, Xq = mxfp8_dequantize(tc, ts), mxfp8_dequantize(xc, xs)
+    dx = np.zeros((R, x.shape[1]), np.float64)
+    dw = np.zeros((E, f2, x.shape[1]), np.float32)
+    p0 = 0
+    for e in range(E):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        plen = (r1 - r0 + 31) // 32 * 32
+        if r1 > r0:
+            wc, ws = mxfp8_quantize(w1[e], axis=1, rounding=0)  # [d, 2f]
+            dx[r0:r1] = gemm_f64(G[r0:r1], mxfp8_dequantize(wc, ws))
+            dw[e] = gemm_f64(Tq[:, p0:p0 + plen], Xq[:, p0:p0 + plen]).astype(np.float32)
+        p0 += plen
+    return {"dx": bf16_from_f64(dx), "dw1": dw if expert_off is not None else dw[0]}
 
 
 def combine(y_bits, pos, w):

@@ -87,3 +87,22 @@ def test_weight_blocks_run_along_the_contraction(orc):
     dx = dgu.astype(np.float64) @ w_expect
     ref_dx = torch.from_numpy(dx).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(r["dx"], ref_dx)
+
+
+def test_grouped_chain_is_per_expert_on_the_grid(orc):
+    """Three experts of 64, 0 and 96 rows: on the grid every expert's dX rows
+    and dW1 are its own fp64 products, and the empty expert's dW1 is zero."""
+    rng = np.random.default_rng(30)
+    off = np.array([0, 64, 64, 160], np.int32)
+    R, f2, d = 160, 64, 96
+    dgu, x = _on_grid(rng, R, f2), _on_grid(rng, R, d)
+    w1 = np.stack([_on_grid(rng, f2, d) for _ in range(3)])
+    r = orc.expert_bwd_gemm1(_bits(dgu), _bits(x), _bits(w1), expert_off=off, seed=3, offset=6)
+    for e in range(3):
+        s = slice(off[e], off[e + 1])
+        dx = dgu[s].astype(np.float64) @ w1[e].astype(np.float64)
+        ref = torch.from_numpy(dx).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(r["dx"][s], ref), e
+        dw = dgu[s].astype(np.float64).T @ x[s].astype(np.float64)
+        assert np.array_equal(r["dw1"][e], dw.astype(np.float32)), e
+    assert not r["dw1"][1].any()
