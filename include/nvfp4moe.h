@@ -315,6 +315,35 @@ nvfp4moe_status swiglu_bwd(const uint16_t *gu, const uint16_t *dh, int64_t rows,
                            uint16_t *dgu, nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * GEMM1 backward in MXFP8 (news.t0001.com '训练数值格式分工清单'; aicoder.com
+ * 'Architecture highlights': MXFP8 backward with stochastic rounding of the
+ * re-quantized gradients). For every expert e, rows [expert_off[e],
+ * expert_off[e+1]) (starts at multiples of 128, as moe_route_permute lays
+ * them out):
+ *   dX_e  = dq(SR(dgu) along 2f)_e . dq(W1_e along 2f)       -> dx bf16 [R x d]
+ *   dW1_e = dq(SR(dgu) along rows)_e^T . dq(RNE(x) along rows)_e -> dw1 fp32 [E x 2f x d]
+ * dgu bf16 [R x 2f] (dg | du, e.g. from swiglu_bwd), x bf16 [R x d]: the
+ *   experts' input rows; rows past expert_off[E] are quantized but never read.
+ * w1t, w1t_sc: W1^T of every expert in MXFP8 with blocks along 2f, codes
+ *   [E*d x 2f] and the MMA layout of its [E*d x 2f/32] scales
+ *   (mxfp8_quantize_sr(W1_e, axis 1, RNE, MMA) per expert).
+ * Stochastic draws: Philox stream (seed, offset) for the row-wise
+ *   quantization of dgu, (seed, offset + 1) for the column-wise one, each
+ *   element at its row-major index in [R x 2f].
+ * Caller-provided intermediates (outputs too), all scales in the MMA layout:
+ *   gq [R x 2f] + gq_sc (dgu along 2f), gt [2f x R] + gt_sc (dgu along rows,
+ *   transposed), xt [d x R] + xt_sc (x along rows, transposed).
+ * R = rows_alloc % 128 == 0, d % 256 == 0, f % 128 == 0, E <= 1024.
+ * Errors: NVFP4MOE_ERR_INVALID_ARG, _SHAPE, _ALIGN before any launch;
+ * NVFP4MOE_ERR_CUDA for a failed launch. */
+nvfp4moe_status moe_expert_bwd_gemm1(const uint16_t *dgu, const uint16_t *x,
+                                     const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
+                                     const uint8_t *w1t, const uint8_t *w1t_sc, uint64_t seed,
+                                     uint64_t offset, uint8_t *gq, uint8_t *gq_sc, uint8_t *gt,
+                                     uint8_t *gt_sc, uint8_t *xt, uint8_t *xt_sc, uint16_t *dx,
+                                     float *dw1, int64_t rows_alloc, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Weighted top-k combine (aicoder.com 'Key Takeaways': the combine step).
  * out[t] = bf16( sum_{j=0..k-1} topk_w[t,j] * y[pos[t,j]] ), fp32 accumulation
  * in slot order with fused multiply-adds; a gather, no atomics.

@@ -412,6 +412,51 @@ nvfp4moe_status swiglu_bwd(const uint16_t *gu, const uint16_t *dh, int64_t rows,
     return after_launch(launch_swiglu_bwd(gu, dh, rows, f, dgu, (cudaStream_t)stream), "swiglu_bwd");
 }
 
+nvfp4moe_status moe_expert_bwd_gemm1(const uint16_t *dgu, const uint16_t *x,
+                                     const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
+                                     const uint8_t *w1t, const uint8_t *w1t_sc, uint64_t seed,
+                                     uint64_t offset, uint8_t *gq, uint8_t *gq_sc, uint8_t *gt,
+                                     uint8_t *gt_sc, uint8_t *xt, uint8_t *xt_sc, uint16_t *dx,
+                                     float *dw1, int64_t rows_alloc, nvfp4moe_stream_t stream) {
+    NEED(E >= 1 && E <= 1024, NVFP4MOE_ERR_INVALID_ARG, "moe_expert_bwd_gemm1: 1 <= E <= 1024");
+    NEED(d > 0 && f > 0 && rows_alloc >= 0, NVFP4MOE_ERR_INVALID_ARG, "moe_expert_bwd_gemm1: sizes");
+    NEED(d % 256 == 0 && f % 128 == 0 && rows_alloc % 128 == 0, NVFP4MOE_ERR_SHAPE,
+         "moe_expert_bwd_gemm1: d %% 256, f %% 128 and rows_alloc %% 128 must be 0");
+    NEED(rows_alloc * (2 * f / 32 + 1) < (1LL << 31) && rows_alloc * (d / 32 + 1) < (1LL << 31),
+         NVFP4MOE_ERR_SHAPE, "moe_expert_bwd_gemm1: tensors too large");
+    NEED_PTR4(expert_off); NEED_PTR(w1t); NEED_PTR(w1t_sc); NEED_PTR(dw1);
+    if (rows_alloc > 0) {
+        NEED_PTR(dgu); NEED_PTR(x); NEED_PTR(gq); NEED_PTR(gq_sc); NEED_PTR(gt); NEED_PTR(gt_sc);
+        NEED_PTR(xt); NEED_PTR(xt_sc); NEED_PTR(dx);
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t R = rows_alloc, f2 = 2 * f;
+    cudaError_t e;
+    // expert starts are multiples of 128, so no 32-row block straddles two experts
+    if ((e = launch_mxfp8_quantize(dgu, R, f2, f2, 0, seed, offset, NVFP4MOE_ROUND_SR, gq, gq_sc,
+                                   NVFP4MOE_LAYOUT_MMA, s)) != cudaSuccess)
+        return cuda_status(e, "moe_expert_bwd_gemm1: quantize dgu rows");
+    if ((e = launch_mxfp8_quantize(dgu, R, f2, f2, 1, seed, offset + 1, NVFP4MOE_ROUND_SR, gt, gt_sc,
+                                   NVFP4MOE_LAYOUT_MMA, s)) != cudaSuccess)
+        return cuda_status(e, "moe_expert_bwd_gemm1: quantize dgu columns");
+    if ((e = launch_mxfp8_quantize(x, R, d, d, 1, 0, 0, NVFP4MOE_ROUND_RNE, xt, xt_sc,
+                                   NVFP4MOE_LAYOUT_MMA, s)) != cudaSuccess)
+        return cuda_status(e, "moe_expert_bwd_gemm1: quantize x columns");
+    GemmArgs g1{};  // dgrad: contraction over 2f, grouped over rows
+    g1.kind = 1; g1.epi = EPI_STORE_BF16; g1.group_axis = NVFP4MOE_GROUP_M;
+    g1.a = gq; g1.a_sc = gq_sc; g1.b = w1t; g1.b_sc = w1t_sc;
+    g1.group_off = expert_off; g1.G = E;
+    g1.a_rows = R; g1.a_cols = f2; g1.M = R; g1.N = d; g1.b_rows_per_group = d; g1.c = dx;
+    if ((e = launch_grouped_gemm(g1, s)) != cudaSuccess) return cuda_status(e, "moe_expert_bwd_gemm1: dgrad");
+    GemmArgs g2{};  // wgrad: contraction over each expert's rows
+    g2.kind = 1; g2.epi = EPI_STORE_F32; g2.group_axis = NVFP4MOE_GROUP_K;
+    g2.a = gt; g2.a_sc = gt_sc; g2.b = xt; g2.b_sc = xt_sc;
+    g2.group_off = expert_off; g2.G = E;
+    g2.a_rows = f2; g2.a_cols = R; g2.M = f2; g2.N = d; g2.b_rows_per_group = d; g2.c = dw1;
+    if ((e = launch_grouped_gemm(g2, s)) != cudaSuccess) return cuda_status(e, "moe_expert_bwd_gemm1: wgrad");
+    return after_launch(cudaSuccess, "moe_expert_bwd_gemm1");
+}
+
 nvfp4moe_status moe_combine(const uint16_t *y, const int32_t *pos, const float *topk_w,
                             int64_t T, int32_t k, int64_t d, uint16_t *out,
                             nvfp4moe_stream_t stream) {

@@ -60,6 +60,8 @@ _SIGS = {
     "moe_expert_fwd_mxfp8": (C.c_int, [_P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _I64, _P]),
     "swiglu_bwd": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
+    "moe_expert_bwd_gemm1": (C.c_int, [_P, _P, _P, _I32, _I64, _I64, _P, _P, _U64, _U64, _P, _P,
+                                       _P, _P, _P, _P, _P, _P, _I64, _P]),
     "moe_combine": (C.c_int, [_P, _P, _P, _I64, _I32, _I64, _P, _P]),
     "moe_combine_rht": (C.c_int, [_P, _P, _P, _I, _U64, _P, _P, _I64, _I32, _I64, _P, _P]),
     "nvfp4_grouped_gemm": (C.c_int, [_P, _P, _P, _I32, _P, _P, _P, _P, _I32, _I64, _I64, _I64, _P,
@@ -223,6 +225,15 @@ def swiglu_bwd(gu, dh, dgu, stream=None):
     """SwiGLU backward: gu [rows, 2f] (g | u), dh [rows, f] -> dgu [rows, 2f] (dg | du), bf16."""
     rows, f = dh.shape
     _check("swiglu_bwd", lib().swiglu_bwd(_ptr(gu), _ptr(dh), rows, f, _ptr(dgu), _stream(stream)))
+
+
+def moe_expert_bwd_gemm1(dgu, x, expert_off, E, d, f, w1t, w1t_sc, seed, offset, gq, gq_sc, gt,
+                         gt_sc, xt, xt_sc, dx, dw1, rows_alloc, stream=None):
+    """GEMM1 backward in MXFP8: dX and dW1 from dgu and x (see include/nvfp4moe.h)."""
+    _check("moe_expert_bwd_gemm1", lib().moe_expert_bwd_gemm1(
+        _ptr(dgu), _ptr(x), _ptr(expert_off), E, d, f, _ptr(w1t), _ptr(w1t_sc), seed, offset,
+        _ptr(gq), _ptr(gq_sc), _ptr(gt), _ptr(gt_sc), _ptr(xt), _ptr(xt_sc), _ptr(dx), _ptr(dw1),
+        rows_alloc, _stream(stream)))
 
 
 def moe_combine(y, pos, topk_w, out, stream=None):

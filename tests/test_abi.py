@@ -85,6 +85,12 @@ P = 1 << 20  # a fake, 16-byte aligned "device pointer"; validation fails before
     (lambda L: L.swiglu_bwd(P, P, 4, 12, P + 4096, None), 2),                         # f % 8
     (lambda L: L.swiglu_bwd(P, P + 4096, 4, 64, P, None), 1),                        # alias
     (lambda L: L.swiglu_bwd(P, P + 8, 4, 64, P + 4096, None), 3),                    # align
+    (lambda L: L.moe_expert_bwd_gemm1(P, P, P, 4, 384, 128, P, P, 0, 0, P, P, P, P, P, P, P, P,
+                                      128, None), 2),                                # d % 256
+    (lambda L: L.moe_expert_bwd_gemm1(P, P, P, 4, 256, 64, P, P, 0, 0, P, P, P, P, P, P, P, P,
+                                      128, None), 2),                                # f % 128
+    (lambda L: L.moe_expert_bwd_gemm1(P, P, P, 4, 256, 128, P, P, 0, 0, P, P, P, None, P, P, P,
+                                      P, 128, None), 1),                             # null gt_sc
     (lambda L: L.moe_combine(P, P, P, 4, 2, 12, P, None), 2),                        # d % 8
     (lambda L: L.nvfp4_grouped_gemm(P, P, P, 2, P, P, P, P, 1, 128, 256, 256, P, 0, None), 1),
     (lambda L: L.nvfp4_grouped_gemm(P, P, P, 0, P, P, P, P, 1, 128, 256, 128, P, 0, None), 2),
