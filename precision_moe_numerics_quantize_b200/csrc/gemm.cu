@@ -761,15 +761,32 @@ bool make_map_swiglu(CUtensorMap *m, const void *base, int64_t E, int64_t f, int
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Grid: two CTAs for every cluster the device keeps resident at once (the
+// Per-device launch set-up, done once per device (a process may drive
+// several GPUs): the shared-memory attribute, the register check, and the
+// grid, two CTAs for every cluster the device keeps resident at once (the
 // tile loop is persistent, so a cluster left waiting for a free pair of SMs
 // would double the tail).
-int pair_grid() {
-    static int n = 0;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        int dev = 0, sms = 0;
-        cudaGetDevice(&dev);
+cudaError_t launch_setup(int &grid) {
+    constexpr int kMaxDevices = 64;
+    static int grids[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (grids[dev] == 0) {
+        e = cudaFuncSetAttribute(grouped_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_ALLOC);
+        if (e != cudaSuccess) return e;
+        // setmaxnreg only redistributes the registers the block launched
+        // with: a build that gave the kernel fewer than REGS_LAUNCH would
+        // leave the epilogue's increase waiting forever
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, grouped_gemm_pair_kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs < (int)REGS_LAUNCH) return cudaErrorInvalidConfiguration;
+        int sms = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (sms <= 1) sms = 148;
         cudaLaunchConfig_t cfg = {};
@@ -782,9 +799,10 @@ int pair_grid() {
             cudaGetLastError();
             clusters = sms / 2;
         }
-        n = 2 * (clusters < sms / 2 ? clusters : sms / 2);
-    });
-    return n;
+        grids[dev] = 2 * (clusters < sms / 2 ? clusters : sms / 2);
+    }
+    grid = grids[dev];
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -831,21 +849,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     if (!okw || !make_map_2d(&mx32, a.a, a.a_rows, kbytes, 32) ||
         !make_map_2d(&mx64, a.a, a.a_rows, kbytes, 64))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-        if (e != cudaSuccess) return e;
-        // setmaxnreg only redistributes the registers the block launched
-        // with: a build that gave the kernel fewer than REGS_LAUNCH would
-        // leave the epilogue's increase waiting forever
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, grouped_gemm_pair_kernel);
-        if (e != cudaSuccess) return e;
-        if (fa.numRegs < (int)REGS_LAUNCH) return cudaErrorInvalidConfiguration;
-        attr_set = true;
-    }
-    grouped_gemm_pair_kernel<<<pair_grid(), NUM_THREADS, SMEM_ALLOC, s>>>(mw, mx32, mx64, p);
+    int grid = 0;
+    cudaError_t e = launch_setup(grid);
+    if (e != cudaSuccess) return e;
+    grouped_gemm_pair_kernel<<<grid, NUM_THREADS, SMEM_ALLOC, s>>>(mw, mx32, mx64, p);
     return cudaGetLastError();
 }
 
