@@ -107,3 +107,40 @@ def test_binding_refuses_cpu_tensors(L):
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         M.nvfp4_quantize(x, x, x, x)
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "nvfp4moe.h"
+int main(void) {
+    if (nvfp4moe_max_rows(16384, 8, 384) != 179840) return 2;
+    /* cols = 48 is not a multiple of 64: rejected on the host, nothing launched */
+    nvfp4moe_status st = nvfp4_quantize((const uint16_t *)0x100000, 4, 48, 48, NULL,
+                                        (uint8_t *)0x100000, (uint8_t *)0x100000,
+                                        (float *)0x100010, NVFP4MOE_LAYOUT_ROWMAJOR, NULL);
+    if (st != NVFP4MOE_ERR_SHAPE) return 3;
+    if (strlen(nvfp4moe_last_error()) == 0) return 4;
+    printf("%s\n", nvfp4moe_last_error());
+    return 0;
+}
+"""
+
+
+def test_plain_c_program_links_and_validates(L, tmp_path):
+    """A C99 program compiled with gcc links against the library and gets the
+    documented status and error text back, with no GPU involved."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "prog.c"
+    src.write_text(C_PROGRAM)
+    libdir = os.path.dirname(M.LIB_PATH)
+    exe = tmp_path / "prog"
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe), f"-L{libdir}", "-l:libnvfp4moe.so",
+                           f"-Wl,-rpath,{libdir}"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert "nvfp4_quantize" in out.stdout
