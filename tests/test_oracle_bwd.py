@@ -69,24 +69,40 @@ def test_ragged_rows_equal_zero_padded_rows(orc):
     assert np.array_equal(r["dw1"], p["dw1"])
 
 
-def test_weight_blocks_run_along_the_contraction(orc):
-    """W1's 32-blocks run along 2f (the dgrad contraction). Column 0 rows 0..31
-    hold 2^18 and values of magnitude <= 1: that block's scale is 2^10, so
-    the small values fall below half the smallest E4M3 step and vanish, while
-    every other block keeps its on-grid values exactly. Blocks along d would
-    flush row 0 instead."""
+def _blocking_case():
     rng = np.random.default_rng(21)
     n, f2, d = 32, 64, 64
     dgu, x, w1 = _on_grid(rng, n, f2), _on_grid(rng, n, d), _on_grid(rng, f2, d)
     small = np.array([0.5, -0.75, 1.0, -0.25], np.float32)
     w1[1:32, 0] = small[np.arange(31) % 4]
     w1[0, 0] = 2.0 ** 18
-    r = orc.expert_bwd_gemm1(_bits(dgu), _bits(x), _bits(w1), seed=2, offset=0)
     w_expect = w1.astype(np.float64)
     w_expect[1:32, 0] = 0.0
     dx = dgu.astype(np.float64) @ w_expect
     ref_dx = torch.from_numpy(dx).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    return dgu, x, w1, ref_dx
+
+
+def test_weight_blocks_run_along_the_contraction(orc):
+    """W1's 32-blocks run along 2f (the dgrad contraction). Column 0 rows 0..31
+    hold 2^18 and values of magnitude <= 1: that block's scale is 2^10, so
+    the small values fall below half the smallest E4M3 step and vanish, while
+    every other block keeps its on-grid values exactly. Blocks along d would
+    flush row 0 instead."""
+    dgu, x, w1, ref_dx = _blocking_case()
+    r = orc.expert_bwd_gemm1(_bits(dgu), _bits(x), _bits(w1), seed=2, offset=0)
     assert np.array_equal(r["dx"], ref_dx)
+
+
+def test_blocking_pin_rejects_weights_blocked_along_d(orc):
+    """The same check fails on a planted copy of the dgrad that blocks W1
+    along d (its rows) instead of along 2f."""
+    dgu, x, w1, ref_dx = _blocking_case()
+    gc, gs = orc.mxfp8_quantize(dgu, axis=0, seed=2, offset=0, rounding=1)
+    wc, ws = orc.mxfp8_quantize(w1, axis=0, rounding=0)  # planted: blocks along d
+    planted = orc.bf16_from_f64(orc.gemm_f64(orc.mxfp8_dequantize(gc, gs),
+                                             orc.mxfp8_dequantize(wc, ws).T.copy()))
+    assert not np.array_equal(planted, ref_dx)
 
 
 def test_grouped_chain_is_per_expert_on_the_grid(orc):
