@@ -20,7 +20,7 @@
  *        stack is fully deterministic).
  *   [P4] 10100.com, "Inkling 2 Small", "PART 01" (384 experts, top-8, 48 layers).
  * None of the pages prints a formula. Every numeric rule below is a reading,
- * marked READING, and the same readings are listed in the design notes.
+ * marked READING at the place it is applied.
  *
  * Precision. Where a floating-point value decides an integer (a quantized
  * code, a scale code, a top-k index) the oracle takes that decision in IEEE
@@ -35,8 +35,14 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <omp.h>
 
 #define ORACLE_API __attribute__((visibility("default")))
+
+/* Threads of the parallel loops (the rows of oracle_gemm_f64). No result
+ * depends on it: the rows are independent and each is summed in order. */
+ORACLE_API void oracle_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
+ORACLE_API int oracle_max_threads(void) { return omp_get_max_threads(); }
 
 /* ------------------------------------------------------------------------ */
 /* bf16                                                                      */
@@ -331,19 +337,22 @@ static void mx_block(const float *vals, const uint64_t *idx, int rounding, uint6
 }
 
 /*
- * x: rows x cols fp32 values (widened bf16), row-major, logical element
- * index i = r * cols + c.
+ * x: rows x cols fp32 values (widened bf16), row-major. Row r of x is row
+ * row0 + r of the source tensor, so the logical element index the stochastic
+ * draws follow is i = (row0 + r) * cols + c (row0 = 0 for a whole tensor;
+ * a larger row0 quantizes a slice of rows with the draws of the whole).
  * axis 0: blocks of 32 along cols. codes [rows x cols], scales [rows x cols/32].
  * axis 1: blocks of 32 along rows inside segments seg_off[0..nseg] (NULL: one
- *   segment of all rows); each segment is zero-padded to a multiple of 32.
+ *   segment of all rows; offsets count rows of x); each segment is
+ *   zero-padded to a multiple of 32.
  *   Output is transposed: codes [cols x Rpad], scales [cols x Rpad/32], where
  *   Rpad is the sum of the padded segment lengths.
  * rounding: 0 = round-to-nearest-even, 1 = stochastic.
  */
-ORACLE_API void oracle_mxfp8_quantize(const float *x, int64_t rows, int64_t cols, int axis,
-                                      const int32_t *seg_off, int32_t nseg, uint64_t seed,
-                                      uint64_t offset, int rounding, uint8_t *codes,
-                                      uint8_t *scales) {
+ORACLE_API void oracle_mxfp8_quantize_at(const float *x, int64_t rows, int64_t cols, int64_t row0,
+                                         int axis, const int32_t *seg_off, int32_t nseg,
+                                         uint64_t seed, uint64_t offset, int rounding,
+                                         uint8_t *codes, uint8_t *scales) {
     float vals[32];
     uint64_t idx[32];
     if (axis == 0) {
@@ -351,7 +360,7 @@ ORACLE_API void oracle_mxfp8_quantize(const float *x, int64_t rows, int64_t cols
             for (int64_t b = 0; b < cols / 32; ++b) {
                 for (int i = 0; i < 32; ++i) {
                     vals[i] = x[r * cols + b * 32 + i];
-                    idx[i] = (uint64_t)(r * cols + b * 32 + i);
+                    idx[i] = (uint64_t)((row0 + r) * cols + b * 32 + i);
                 }
                 mx_block(vals, idx, rounding, seed, offset, codes + r * cols + b * 32, 1,
                          scales + r * (cols / 32) + b);
@@ -371,7 +380,7 @@ ORACLE_API void oracle_mxfp8_quantize(const float *x, int64_t rows, int64_t cols
                 for (int i = 0; i < 32; ++i) {
                     int64_t r = r0 + b * 32 + i;
                     vals[i] = (r < r1) ? x[r * cols + c] : 0.0f;
-                    idx[i] = (r < r1) ? (uint64_t)(r * cols + c) : 0;
+                    idx[i] = (r < r1) ? (uint64_t)((row0 + r) * cols + c) : 0;
                 }
                 mx_block(vals, idx, rounding, seed, offset, codes + c * Rpad + out_r + b * 32, 1,
                          scales + c * (Rpad / 32) + (out_r / 32) + b);
@@ -379,6 +388,14 @@ ORACLE_API void oracle_mxfp8_quantize(const float *x, int64_t rows, int64_t cols
         }
         out_r += len;
     }
+}
+
+ORACLE_API void oracle_mxfp8_quantize(const float *x, int64_t rows, int64_t cols, int axis,
+                                      const int32_t *seg_off, int32_t nseg, uint64_t seed,
+                                      uint64_t offset, int rounding, uint8_t *codes,
+                                      uint8_t *scales) {
+    oracle_mxfp8_quantize_at(x, rows, cols, 0, axis, seg_off, nseg, seed, offset, rounding, codes,
+                             scales);
 }
 
 /* x_hat = e4m3(q) * 2^(e - 127), exact. layout as produced above with
@@ -461,6 +478,20 @@ ORACLE_API void oracle_rht32_f64(const double *x, uint32_t signs, int inverse, d
         double u = t[i] * c;
         y[i] = (inverse && ((signs >> i) & 1)) ? -u : u;
     }
+}
+
+/* max |v| over the RHT32 transform v of rows x cols values: the tensor amax an
+ * NVFP4 payload takes, computed a slice of rows at a time for large tensors. */
+ORACLE_API float oracle_rht32_amax(const float *x, int64_t rows, int64_t cols, uint64_t sign_seed) {
+    uint32_t s = oracle_rht_signs(sign_seed);
+    float v[32], amax = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < cols / 32; ++b) {
+            oracle_rht32_forward_f32(x + r * cols + b * 32, s, v);
+            for (int i = 0; i < 32; ++i)
+                if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+        }
+    return amax;
 }
 
 /*

@@ -17,7 +17,7 @@ __all__ = [
     "rht_signs", "rht32_forward_f32", "rht32_inverse_f32", "rht32_f64", "rht32_quantize",
     "rht32_dequantize", "route", "permute", "gemm_f64", "swiglu", "expert_ffn", "combine",
     "combine_f32", "combine_rht", "mxfp8_rpad", "expert_ffn_mxfp8", "swiglu_bwd",
-    "expert_bwd_gemm1",
+    "expert_bwd_gemm1", "set_threads", "max_threads", "rht32_amax",
 ]
 
 _lib = None
@@ -39,6 +39,8 @@ _U64 = C.c_uint64
 
 def _declare(L):
     sig = {
+        "oracle_set_threads": (None, [C.c_int]),
+        "oracle_max_threads": (C.c_int, []),
         "oracle_bf16_to_f32": (C.c_float, [C.c_uint16]),
         "oracle_bf16_from_f64": (C.c_uint16, [C.c_double]),
         "oracle_e2m1_decode": (C.c_double, [C.c_uint8]),
@@ -54,6 +56,9 @@ def _declare(L):
         "oracle_philox_word": (C.c_uint32, [_U64, _U64, _U64]),
         "oracle_mxfp8_quantize": (None, [_P, _I64, _I64, C.c_int, _P, _I32, _U64, _U64, C.c_int,
                                          _P, _P]),
+        "oracle_mxfp8_quantize_at": (None, [_P, _I64, _I64, _I64, C.c_int, _P, _I32, _U64, _U64,
+                                            C.c_int, _P, _P]),
+        "oracle_rht32_amax": (C.c_float, [_P, _I64, _I64, _U64]),
         "oracle_mxfp8_dequantize": (None, [_P, _P, _I64, _I64, _P]),
         "oracle_rht_signs": (C.c_uint32, [_U64]),
         "oracle_rht32_forward_f32": (None, [_P, C.c_uint32, _P]),
@@ -180,9 +185,11 @@ def mxfp8_rpad(seg_off, rows):
     return int(sum((int(s[i + 1] - s[i]) + 31) // 32 * 32 for i in range(len(s) - 1)))
 
 
-def mxfp8_quantize(x, axis=0, seg_off=None, seed=0, offset=0, rounding=0):
+def mxfp8_quantize(x, axis=0, seg_off=None, seed=0, offset=0, rounding=0, row0=0):
     """Returns (codes, scales). axis 0: [rows, cols], [rows, cols/32].
-    axis 1: transposed [cols, Rpad], [cols, Rpad/32]."""
+    axis 1: transposed [cols, Rpad], [cols, Rpad/32]. row0: the first row's
+    index in the source tensor (the stochastic draws follow the source's
+    row-major element index)."""
     x = _c(x, np.float32)
     rows, cols = x.shape
     if axis == 0:
@@ -195,8 +202,8 @@ def mxfp8_quantize(x, axis=0, seg_off=None, seed=0, offset=0, rounding=0):
         scales = np.zeros((cols, rp // 32), np.uint8)
         so = None if seg_off is None else _c(seg_off, np.int32)
         ns = 0 if seg_off is None else len(seg_off) - 1
-    lib().oracle_mxfp8_quantize(_p(x), rows, cols, axis, _p(so), ns, seed, offset, rounding,
-                                _p(codes), _p(scales))
+    lib().oracle_mxfp8_quantize_at(_p(x), rows, cols, int(row0), axis, _p(so), ns, seed, offset,
+                                   rounding, _p(codes), _p(scales))
     return codes, scales
 
 
@@ -441,3 +448,19 @@ def combine_f32(y, pos, w):
     out = np.zeros((T, d), np.uint16)
     lib().oracle_combine_f32(_p(y), _p(pos), _p(w), T, k, d, _p(out))
     return out
+
+
+def set_threads(n):
+    """Threads of the oracle's parallel loops (results do not depend on it)."""
+    lib().oracle_set_threads(int(n))
+
+
+def max_threads():
+    return int(lib().oracle_max_threads())
+
+
+def rht32_amax(x, sign_seed):
+    """max |v| of the RHT32 transform of x [rows, cols] (fp32 values)."""
+    x = _c(x, np.float32)
+    rows, cols = x.shape
+    return np.float32(lib().oracle_rht32_amax(_p(x), rows, cols, sign_seed))

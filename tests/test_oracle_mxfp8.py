@@ -135,3 +135,33 @@ def test_axis1_segments_pad_with_zeros(orc):
     xa[:20] = x[:20]
     ca, sa = orc.mxfp8_quantize(xa, axis=1, rounding=0)
     assert np.array_equal(c[:, :32], ca) and np.array_equal(s[:, :1], sa)
+
+
+def test_row_offset_keeps_the_source_element_index(orc):
+    """A slice of rows quantized with row0 = its first row's index gives the
+    whole tensor's codes for those rows, and each stochastic decision follows
+    the Philox word of the element's row-major index in the whole tensor."""
+    rows, cols, r0, r1 = 96, 64, 32, 80
+    x = _x(rows, cols, 8) * np.float32(0.05)
+    full = orc.mxfp8_quantize(x, seed=7, offset=2, rounding=1)
+    part = orc.mxfp8_quantize(x[r0:r1], seed=7, offset=2, rounding=1, row0=r0)
+    assert np.array_equal(part[0], full[0][r0:r1]) and np.array_equal(part[1], full[1][r0:r1])
+    # axis 1: the 32-row blocks of rows 32..95 are columns 32..95 of the whole
+    full1 = orc.mxfp8_quantize(x, axis=1, seed=7, offset=3, rounding=1)
+    part1 = orc.mxfp8_quantize(x[32:96], axis=1, seed=7, offset=3, rounding=1, row0=32)
+    assert np.array_equal(part1[0], full1[0][:, 32:96])
+    # explicit decisions: round up iff (word >> 8) * 2^-24 < the fraction of
+    # the way from the lower E4M3 neighbour to the upper one
+    k = np.repeat(part[1].astype(np.int64) - 127, 32, axis=1)
+    v = np.abs(x[r0:r1].astype(np.float64) * 2.0 ** (-k))
+    g = np.array(_e4m3_grid())
+    lo = g[np.searchsorted(g, v, side="right") - 1]
+    hi = g[np.minimum(np.searchsorted(g, v, side="left"), len(g) - 1)]
+    got = np.abs(orc.mxfp8_dequantize(part[0], part[1]).astype(np.float64) * 2.0 ** (-k))
+    for r in range(r1 - r0):
+        for c in range(cols):
+            if lo[r, c] == hi[r, c]:
+                continue
+            wd = orc.philox_word(7, 2, (r0 + r) * cols + c)
+            up = (wd >> 8) * 2.0 ** -24 < (v[r, c] - lo[r, c]) / (hi[r, c] - lo[r, c])
+            assert got[r, c] == (hi[r, c] if up else lo[r, c]), (r, c)

@@ -175,3 +175,20 @@ def test_combine_rht_is_the_combine_of_the_inverted_rows(orc):
         assert np.abs(via_rows - once).max() <= 2 ** -8 * mag
         # and the two agree to the last bit on most elements
         assert np.mean(via_rows == once) > 0.9
+
+
+def test_rht32_amax_is_max_of_the_transform(orc):
+    """The payload amax helper equals max |v| of the transform written out with
+    scipy's Hadamard matrix in fp64, to the fp32 evaluation's rounding bound,
+    and the NVFP4 payload's tensor scale is that amax / 2688."""
+    x = synth.bf16_bits_to_f32(synth.payload_rows_np(5, 0, 16, 128, synth.outlier_channels(5, 128, 4)))
+    s = orc.rht_signs(11)
+    D = np.array([-1.0 if (s >> i) & 1 else 1.0 for i in range(32)])
+    H = scipy.linalg.hadamard(32).astype(np.float64) / np.sqrt(32.0)
+    v = (x.astype(np.float64).reshape(16, 4, 32) * D) @ H.T
+    am = orc.rht32_amax(x, 11)
+    ref = np.abs(v).max()
+    bound = 5 * 2.0 ** -24 * np.abs(x.astype(np.float64).reshape(16, 4, 32)).sum(axis=2).max()
+    assert abs(float(am) - ref) <= bound
+    _, _, ts = orc.rht32_quantize(x, 11, 0)
+    assert ts == np.float32(am / np.float32(2688.0))
