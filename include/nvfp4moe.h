@@ -44,8 +44,9 @@
  *   - Every call is asynchronous on the given stream, performs no host
  *     synchronisation, and is deterministic (identical bits for identical
  *     inputs). The one piece of library state is a device-side error word
- *     set by a kernel whose bounded wait ran out; nvfp4moe_device_error()
- *     reads and clears it.
+ *     set by a kernel whose bounded wait ran out or that found device-side
+ *     arguments it could not use; nvfp4moe_device_error() reads and clears
+ *     it.
  *   - bf16 tensors are passed as uint16_t bit patterns, row-major, with a row
  *     stride ld in elements (ld >= cols, ld % 8 == 0).
  *   - NVFP4 codes: rows x cols/2 bytes, element 2i in the low nibble of byte i.
@@ -100,9 +101,24 @@ int nvfp4moe_version(void);
 const char *nvfp4moe_last_error(void);
 
 /* Synchronises the current device, then reads and clears the device error
- * word. *code (host) receives 0 if no kernel gave up a bounded wait, else the
- * identifier of the wait that ran out. Returns NVFP4MOE_ERR_TIMEOUT if set. */
+ * word. *code (host) receives 0 if no kernel recorded an error, 1..15 for the
+ * identifier of a bounded GEMM wait that ran out (returns
+ * NVFP4MOE_ERR_TIMEOUT), or NVFP4MOE_DEVERR_SEGMENTS if mxfp8_quantize_sr was
+ * given segment offsets that are not non-decreasing inside [0, rows]
+ * (returns NVFP4MOE_ERR_INVALID_ARG). */
+enum { NVFP4MOE_DEVERR_SEGMENTS = 16 };
 nvfp4moe_status nvfp4moe_device_error(int32_t *code);
+
+/* Test hook of the failure path of the grouped GEMMs (no counterpart on the
+ * pages). flags = NVFP4MOE_DEBUG_WITHHOLD_LOADS makes the GEMM launches that
+ * follow (in this process) issue no operand or scale load at all, so no copy
+ * is ever in flight; their consumers' bounded waits then give up after
+ * wait_ns nanoseconds (0: the normal 2 s), every role winds down, the launch
+ * ends, and nvfp4moe_device_error() reports NVFP4MOE_ERR_TIMEOUT with the id
+ * of the wait that gave up first. flags = 0 restores normal operation (and
+ * the 2 s limit). Not for use while other threads launch GEMMs. */
+enum { NVFP4MOE_DEBUG_WITHHOLD_LOADS = 1 };
+nvfp4moe_status nvfp4moe_debug_gemm(uint32_t flags, uint64_t wait_ns);
 
 /* Exhaustive check of the hardware conversions the kernels use against the
  * library's own encoders and decoders (which the test suite pins bit for bit
@@ -152,17 +168,34 @@ nvfp4moe_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, co
  * x: bf16 [rows x cols], stride ld.
  * axis 0: blocks of 32 along a row. cols % 32 == 0 (MMA layout: rows % 128,
  *   cols % 128). codes [rows x cols], scales E8M0 [rows x cols/32].
- * axis 1: blocks of 32 consecutive rows of a column; rows % 32 == 0 (MMA:
- *   rows % 128, cols % 128). The output is transposed, ready to be the
- *   K-major operand of a GEMM that contracts over rows: codes [cols x rows],
- *   scales [cols x rows/32]. To keep blocks inside expert segments, start
- *   every segment on a 32-row boundary (moe_route_permute pads to 128).
+ * axis 1: blocks of 32 consecutive rows of a column, cols % 64 == 0. The
+ *   output is transposed, ready to be the K-major operand of a GEMM that
+ *   contracts over rows.
+ *   seg_off == NULL: one segment of all rows; rows % 32 == 0 (MMA: rows %
+ *     128, cols % 128); codes [cols x rows], scales [cols x rows/32].
+ *   seg_off != NULL: device int32 [nseg + 1], 1 <= nseg <= 1024,
+ *     non-decreasing inside [0, rows]; segment s is rows [seg_off[s],
+ *     seg_off[s+1]). No block crosses a segment: each segment is cut into
+ *     ceil(len / 32) blocks, the last one zero-padded, and the blocks of all
+ *     segments are packed in order into an output of
+ *     P = nvfp4moe_mxfp8_seg_rows(rows, nseg) columns (the most the packed
+ *     blocks can need): codes [cols x P], scales [cols x P/32]; columns past
+ *     the packed blocks get zero codes and zero scale codes (MMA layout: P %
+ *     128 and cols % 128). The offsets are checked on the device: invalid
+ *     ones give an all-zero output and NVFP4MOE_DEVERR_SEGMENTS in the device
+ *     error word (nvfp4moe_device_error).
  * rounding: NVFP4MOE_ROUND_RNE or NVFP4MOE_ROUND_SR (seed, offset select the
- *   Philox stream; quantize the same tensor along two axes with two offsets). */
+ *   Philox stream; quantize the same tensor along two axes with two offsets).
+ *   A draw follows the element's row-major index in the [rows x cols] source,
+ *   with or without segments. */
 nvfp4moe_status mxfp8_quantize_sr(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                                  int axis, uint64_t seed, uint64_t offset, int rounding,
-                                  uint8_t *codes, uint8_t *scales, int layout,
-                                  nvfp4moe_stream_t stream);
+                                  int axis, const int32_t *seg_off, int32_t nseg, uint64_t seed,
+                                  uint64_t offset, int rounding, uint8_t *codes, uint8_t *scales,
+                                  int layout, nvfp4moe_stream_t stream);
+
+/* Output columns of a segmented column-wise MXFP8 quantization:
+ * round_up(rows + 31 * nseg, 32); -1 for rows < 0 or nseg < 1. */
+int64_t nvfp4moe_mxfp8_seg_rows(int64_t rows, int32_t nseg);
 
 /* out = e4m3(code) * 2^(scale - 127), fp32 [n_rows x n_cols] for an MXFP8
  * tensor stored as codes [n_rows x n_cols] with ROWMAJOR or MMA scales. */
@@ -260,7 +293,9 @@ nvfp4moe_status moe_route_permute_noalloc(const float *logits, const uint16_t *x
  * Caller-provided intermediates (outputs too): h bf16 [R x f], hq [R x f/2],
  *   hq_sc MMA layout of [R x f], h_amax fp32 [E], h_ts fp32 [E].
  * y bf16 [R x d]. R = rows_alloc >= expert_off[E], R % 128 == 0.
- * d % 256 == 0, f % 256 == 0, E <= 1024. */
+ * d % 256 == 0, f % 256 == 0, E <= 1024.
+ * Three kernel launches: GEMM1 with SwiGLU and the amax of h, the grouped
+ * requantization of h, GEMM2. */
 nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const float *x_ts,
                                const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
                                const uint8_t *w1, const uint8_t *w1_sc, const float *w1_ts,
@@ -268,6 +303,24 @@ nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const fl
                                uint16_t *h, uint8_t *hq, uint8_t *hq_sc, float *h_amax,
                                float *h_ts, uint16_t *y, int64_t rows_alloc,
                                nvfp4moe_stream_t stream);
+
+/* The same expert FFN with the requantization of h fused into GEMM1 (the
+ * pages' re-quantization step kept inside the first GEMM's launch: aicoder.com
+ * 'Key Takeaways'): every expert is published once its last tile is stored
+ * and its rows are requantized by the epilogue warps when their tiles are
+ * done, while much of h is still in L2; two kernel launches. Same arguments
+ * and results (bit for bit) as moe_expert_fwd, plus ws: a device workspace of
+ * at least moe_expert_fwd_fused_requant_workspace_size(E) bytes (16-byte
+ * aligned, a few KB), cleared by the call itself (NVFP4MOE_ERR_WORKSPACE if
+ * smaller). On B200 it is slower than moe_expert_fwd, which is therefore the
+ * default path. */
+size_t moe_expert_fwd_fused_requant_workspace_size(int32_t E);
+nvfp4moe_status moe_expert_fwd_fused_requant(
+    const uint8_t *xq, const uint8_t *xq_sc, const float *x_ts, const int32_t *expert_off,
+    int32_t E, int64_t d, int64_t f, const uint8_t *w1, const uint8_t *w1_sc, const float *w1_ts,
+    const uint8_t *w2, const uint8_t *w2_sc, const float *w2_ts, uint16_t *h, uint8_t *hq,
+    uint8_t *hq_sc, float *h_amax, float *h_ts, uint16_t *y, int64_t rows_alloc, void *ws,
+    size_t ws_bytes, nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Expert FFN forward in MXFP8 (aicoder.com 'Architecture highlights': the last

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "quant.cuh"
@@ -24,6 +25,48 @@ nvfp4moe_status cuda_status(cudaError_t e, const char *what) {
     if (e == cudaSuccess) return NVFP4MOE_OK;
     set_last_error("%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
     return NVFP4MOE_ERR_CUDA;
+}
+
+// The current driver context (nullptr if the driver entry point is missing).
+// A __device__ variable's address belongs to the module loaded in one
+// context: a reset device, or another context made current on the same
+// device, loads the module again and the variable can move.
+static void *current_context() {
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    static GetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &ptr, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCurrentFn>(ptr);
+    });
+    CUcontext c = nullptr;
+    if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+}
+
+cudaError_t cached_symbol_address(SymbolAddressCache &cache, const void *symbol, void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    void *ctx = current_context();
+    std::lock_guard<std::mutex> lock(cache.mu);
+    for (int i = 0; i < cache.n; ++i)
+        if (cache.entry[i].dev == dev && cache.entry[i].ctx == ctx) {
+            *out = cache.entry[i].addr;
+            return cudaSuccess;
+        }
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, symbol);
+    if (e != cudaSuccess) return e;
+    // a full table is recycled from the start: a miss only costs a lookup
+    const int slot = cache.n < SymbolAddressCache::kEntries ? cache.n++ : (cache.next++ % cache.n);
+    cache.entry[slot] = {dev, ctx, p};
+    *out = p;
+    return cudaSuccess;
 }
 
 }  // namespace nvfp4moe
@@ -125,6 +168,8 @@ nvfp4moe_status nvfp4moe_device_error(int32_t *code) {
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_status(e, "nvfp4moe_device_error: read");
     *code = v;
+    if (v == NVFP4MOE_DEVERR_SEGMENTS)
+        FAIL(NVFP4MOE_ERR_INVALID_ARG, "mxfp8_quantize_sr: segment offsets not non-decreasing in [0, rows]");
     if (v) FAIL(NVFP4MOE_ERR_TIMEOUT, "a bounded device wait ran out (wait id %d)", v);
     return NVFP4MOE_OK;
 }
@@ -201,16 +246,42 @@ nvfp4moe_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, co
         "nvfp4_dequantize");
 }
 
+int64_t nvfp4moe_mxfp8_seg_rows(int64_t rows, int32_t nseg) {
+    if (rows < 0 || nseg < 1) return -1;
+    return (rows + 31 * (int64_t)nseg + 31) / 32 * 32;
+}
+
 nvfp4moe_status mxfp8_quantize_sr(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                                  int axis, uint64_t seed, uint64_t offset, int rounding,
-                                  uint8_t *codes, uint8_t *scales, int layout,
-                                  nvfp4moe_stream_t stream) {
+                                  int axis, const int32_t *seg_off, int32_t nseg, uint64_t seed,
+                                  uint64_t offset, int rounding, uint8_t *codes, uint8_t *scales,
+                                  int layout, nvfp4moe_stream_t stream) {
     NEED(rows >= 0 && cols >= 0, NVFP4MOE_ERR_INVALID_ARG, "mxfp8_quantize_sr: negative size");
     NEED(axis == 0 || axis == 1, NVFP4MOE_ERR_INVALID_ARG, "mxfp8_quantize_sr: axis must be 0 or 1");
     NEED(rounding == NVFP4MOE_ROUND_RNE || rounding == NVFP4MOE_ROUND_SR,
          NVFP4MOE_ERR_INVALID_ARG, "mxfp8_quantize_sr: bad rounding %d", rounding);
     NEED(ld % 8 == 0 && ld >= cols, NVFP4MOE_ERR_SHAPE, "mxfp8_quantize_sr: ld %% 8 == 0, ld >= cols");
     NEED(rows * (cols / 32 + 1) < (1LL << 31), NVFP4MOE_ERR_SHAPE, "mxfp8_quantize_sr: tensor too large");
+    if (seg_off) {
+        NEED(axis == 1, NVFP4MOE_ERR_INVALID_ARG, "mxfp8_quantize_sr: segments need axis 1");
+        NEED(nseg >= 1 && nseg <= 1024, NVFP4MOE_ERR_INVALID_ARG,
+             "mxfp8_quantize_sr: 1 <= nseg <= 1024 (got %d)", nseg);
+        NEED_PTR4(seg_off);
+        NEED(cols % 64 == 0, NVFP4MOE_ERR_SHAPE, "mxfp8_quantize_sr: axis 1 needs cols %% 64 == 0");
+        const int64_t pitch = nvfp4moe_mxfp8_seg_rows(rows, nseg);
+        NEED(pitch * (cols / 32 + 1) < (1LL << 31), NVFP4MOE_ERR_SHAPE,
+             "mxfp8_quantize_sr: tensor too large");
+        nvfp4moe_status st = check_layout(layout, cols, pitch / 32, "mxfp8_quantize_sr");
+        if (st) return st;
+        if (pitch * cols) {
+            if (rows * cols) NEED_PTR(x);
+            NEED_PTR(codes);
+            NEED_PTR(scales);
+        }
+        return after_launch(launch_mxfp8_quantize_seg(x, rows, cols, ld, seg_off, nseg, pitch, seed,
+                                                      offset, rounding, codes, scales, layout,
+                                                      (cudaStream_t)stream),
+                            "mxfp8_quantize_sr");
+    }
     if (axis == 0) {
         NEED(cols % 32 == 0, NVFP4MOE_ERR_SHAPE, "mxfp8_quantize_sr: axis 0 needs cols %% 32 == 0");
         nvfp4moe_status st = check_layout(layout, rows, cols / 32, "mxfp8_quantize_sr");
@@ -322,24 +393,39 @@ nvfp4moe_status moe_route_permute(const float *logits, const uint16_t *x, int64_
                         "moe_route_permute");
 }
 
-nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const float *x_ts,
-                               const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
-                               const uint8_t *w1, const uint8_t *w1_sc, const float *w1_ts,
-                               const uint8_t *w2, const uint8_t *w2_sc, const float *w2_ts,
-                               uint16_t *h, uint8_t *hq, uint8_t *hq_sc, float *h_amax,
-                               float *h_ts, uint16_t *y, int64_t rows_alloc,
-                               nvfp4moe_stream_t stream) {
-    NEED(E >= 1 && E <= 1024, NVFP4MOE_ERR_INVALID_ARG, "moe_expert_fwd: 1 <= E <= 1024");
-    NEED(d > 0 && f > 0 && rows_alloc >= 0, NVFP4MOE_ERR_INVALID_ARG, "moe_expert_fwd: sizes");
-    NEED(d % 256 == 0 && f % 256 == 0 && rows_alloc % 128 == 0, NVFP4MOE_ERR_SHAPE,
-         "moe_expert_fwd: d %% 256, f %% 256 and rows_alloc %% 128 must be 0");
+nvfp4moe_status nvfp4moe_debug_gemm(uint32_t flags, uint64_t wait_ns) {
+    NEED((flags & ~1u) == 0, NVFP4MOE_ERR_INVALID_ARG, "nvfp4moe_debug_gemm: unknown flags 0x%x", flags);
+    set_gemm_debug(flags, wait_ns);
+    return NVFP4MOE_OK;
+}
+
+// The NVFP4 expert FFN; with ws == nullptr the requantization of h is its
+// own kernel between the GEMMs, otherwise it is fused into GEMM1.
+static nvfp4moe_status expert_fwd(const char *fn, const uint8_t *xq, const uint8_t *xq_sc,
+                                  const float *x_ts, const int32_t *expert_off, int32_t E,
+                                  int64_t d, int64_t f, const uint8_t *w1, const uint8_t *w1_sc,
+                                  const float *w1_ts, const uint8_t *w2, const uint8_t *w2_sc,
+                                  const float *w2_ts, uint16_t *h, uint8_t *hq, uint8_t *hq_sc,
+                                  float *h_amax, float *h_ts, uint16_t *y, int64_t rows_alloc,
+                                  void *ws, size_t ws_bytes, bool fused, cudaStream_t s) {
+    if (!(E >= 1 && E <= 1024)) FAIL(NVFP4MOE_ERR_INVALID_ARG, "%s: 1 <= E <= 1024", fn);
+    if (!(d > 0 && f > 0 && rows_alloc >= 0)) FAIL(NVFP4MOE_ERR_INVALID_ARG, "%s: sizes", fn);
+    if (!(d % 256 == 0 && f % 256 == 0 && rows_alloc % 128 == 0))
+        FAIL(NVFP4MOE_ERR_SHAPE, "%s: d %% 256, f %% 256 and rows_alloc %% 128 must be 0", fn);
     NEED_PTR(xq); NEED_PTR(xq_sc); NEED_PTR4(x_ts); NEED_PTR4(expert_off);
     NEED_PTR(w1); NEED_PTR(w1_sc); NEED_PTR4(w1_ts);
     NEED_PTR(w2); NEED_PTR(w2_sc); NEED_PTR4(w2_ts);
     NEED_PTR(h); NEED_PTR(hq); NEED_PTR(hq_sc); NEED_PTR4(h_amax); NEED_PTR4(h_ts); NEED_PTR(y);
-    cudaStream_t s = (cudaStream_t)stream;
+    const size_t need = requant_ws_bytes(E);
+    if (fused) {
+        if (!ws || ws_bytes < need)
+            FAIL(NVFP4MOE_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                 ws ? ws_bytes : (size_t)0);
+        NEED_PTR(ws);
+    }
     cudaError_t e = cudaMemsetAsync(h_amax, 0, sizeof(float) * E, s);
-    if (e != cudaSuccess) return cuda_status(e, "moe_expert_fwd: memset");
+    if (e == cudaSuccess && fused) e = cudaMemsetAsync(ws, 0, need, s);
+    if (e != cudaSuccess) return cuda_status(e, fn);
     GemmArgs g1{};
     g1.kind = 0; g1.epi = EPI_SWIGLU_AMAX; g1.group_axis = NVFP4MOE_GROUP_M;
     g1.a = xq; g1.a_sc = xq_sc; g1.a_ts = x_ts; g1.a_ts_stride = 0;
@@ -347,10 +433,13 @@ nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const fl
     g1.group_off = expert_off; g1.G = E;
     g1.a_rows = rows_alloc; g1.a_cols = d; g1.N = 2 * f; g1.b_rows_per_group = 2 * f;
     g1.c = h; g1.amax = h_amax;
-    if ((e = launch_grouped_gemm(g1, s)) != cudaSuccess) return cuda_status(e, "moe_expert_fwd: gemm1");
-    if ((e = launch_nvfp4_quant_grouped(h, rows_alloc, f, expert_off, E, h_amax, hq, hq_sc, h_ts,
-                                        s)) != cudaSuccess)
-        return cuda_status(e, "moe_expert_fwd: requantize");
+    if (fused) {
+        g1.hq = hq; g1.hq_sc = hq_sc; g1.h_ts = h_ts; g1.rq_ws = ws;
+    }
+    if ((e = launch_grouped_gemm(g1, s)) != cudaSuccess) return cuda_status(e, fn);
+    if (!fused && (e = launch_nvfp4_quant_grouped(h, rows_alloc, f, expert_off, E, h_amax, hq,
+                                                  hq_sc, h_ts, s)) != cudaSuccess)
+        return cuda_status(e, fn);
     GemmArgs g2{};
     g2.kind = 0; g2.epi = EPI_STORE_BF16; g2.group_axis = NVFP4MOE_GROUP_M;
     g2.a = hq; g2.a_sc = hq_sc; g2.a_ts = h_ts; g2.a_ts_stride = 1;
@@ -358,8 +447,35 @@ nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const fl
     g2.group_off = expert_off; g2.G = E;
     g2.a_rows = rows_alloc; g2.a_cols = f; g2.N = d; g2.b_rows_per_group = d;
     g2.c = y;
-    if ((e = launch_grouped_gemm(g2, s)) != cudaSuccess) return cuda_status(e, "moe_expert_fwd: gemm2");
-    return after_launch(cudaSuccess, "moe_expert_fwd");
+    if ((e = launch_grouped_gemm(g2, s)) != cudaSuccess) return cuda_status(e, fn);
+    return after_launch(cudaSuccess, fn);
+}
+
+nvfp4moe_status moe_expert_fwd(const uint8_t *xq, const uint8_t *xq_sc, const float *x_ts,
+                               const int32_t *expert_off, int32_t E, int64_t d, int64_t f,
+                               const uint8_t *w1, const uint8_t *w1_sc, const float *w1_ts,
+                               const uint8_t *w2, const uint8_t *w2_sc, const float *w2_ts,
+                               uint16_t *h, uint8_t *hq, uint8_t *hq_sc, float *h_amax,
+                               float *h_ts, uint16_t *y, int64_t rows_alloc,
+                               nvfp4moe_stream_t stream) {
+    return expert_fwd("moe_expert_fwd", xq, xq_sc, x_ts, expert_off, E, d, f, w1, w1_sc, w1_ts, w2,
+                      w2_sc, w2_ts, h, hq, hq_sc, h_amax, h_ts, y, rows_alloc, nullptr, 0, false,
+                      (cudaStream_t)stream);
+}
+
+size_t moe_expert_fwd_fused_requant_workspace_size(int32_t E) {
+    return E < 0 ? 0 : requant_ws_bytes(E);
+}
+
+nvfp4moe_status moe_expert_fwd_fused_requant(
+    const uint8_t *xq, const uint8_t *xq_sc, const float *x_ts, const int32_t *expert_off,
+    int32_t E, int64_t d, int64_t f, const uint8_t *w1, const uint8_t *w1_sc, const float *w1_ts,
+    const uint8_t *w2, const uint8_t *w2_sc, const float *w2_ts, uint16_t *h, uint8_t *hq,
+    uint8_t *hq_sc, float *h_amax, float *h_ts, uint16_t *y, int64_t rows_alloc, void *ws,
+    size_t ws_bytes, nvfp4moe_stream_t stream) {
+    return expert_fwd("moe_expert_fwd_fused_requant", xq, xq_sc, x_ts, expert_off, E, d, f, w1,
+                      w1_sc, w1_ts, w2, w2_sc, w2_ts, h, hq, hq_sc, h_amax, h_ts, y, rows_alloc, ws,
+                      ws_bytes, true, (cudaStream_t)stream);
 }
 
 nvfp4moe_status moe_expert_fwd_mxfp8(const uint8_t *xq, const uint8_t *xq_sc,

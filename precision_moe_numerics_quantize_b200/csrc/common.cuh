@@ -9,6 +9,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/nvfp4moe.h"
 
 #define NV_DEV __device__ __forceinline__
@@ -20,6 +22,22 @@ namespace nvfp4moe {
 // ---------------------------------------------------------------------------
 void set_last_error(const char *fmt, ...);
 nvfp4moe_status cuda_status(cudaError_t e, const char *what);
+
+// Device addresses of a __device__ variable, one per (device, driver context)
+// the library has run in: looked up with cudaGetSymbolAddress on the first
+// call in that device and context, then reused.
+struct SymbolAddressCache {
+    static constexpr int kEntries = 64;
+    struct Entry {
+        int dev;
+        void *ctx;
+        void *addr;
+    };
+    std::mutex mu;
+    Entry entry[kEntries];
+    int n = 0, next = 0;
+};
+cudaError_t cached_symbol_address(SymbolAddressCache &cache, const void *symbol, void **out);
 
 // Device error word: a kernel whose bounded wait ran out stores the id of the
 // wait here (first writer wins) and returns early.
@@ -37,6 +55,9 @@ enum WaitId : int32_t {
     WAIT_GEMM_SF_SLOT = 6,
     WAIT_GEMM_SF_FULL = 7,
     WAIT_GEMM_SF_FREE = 8,
+    // not a wait: a kernel found device-side arguments it could not use
+    DEVERR_SEGMENTS = NVFP4MOE_DEVERR_SEGMENTS,  // mxfp8 columns: bad segment offsets
+    DEVERR_REQUANT = 17,  // fused requantization: a queue entry outside its expert
 };
 
 // ---------------------------------------------------------------------------

@@ -21,11 +21,10 @@
 // protocol allows.
 //
 // Roles (640 threads, 20 warps, in both CTAs of the pair):
-//   warp 0       TMA producer: this CTA's W and X halves (128-byte swizzle),
-//                completion counted on the first CTA's `full` barrier, and
-//                the X block scales of the stage (plain bulk copies of the one
-//                or two 128-row chunk rows) into this CTA: counted on `full`
-//                in the first CTA, on its own `sf_loaded` in the other.
+//   warp 0       TMA producer: first the X block scales of the stage (plain
+//                bulk copies of the one or two 128-row chunk rows) into this
+//                CTA, counted on its own `sf_loaded`; then this CTA's W and X
+//                halves (128-byte swizzle), counted on the first CTA's `full`.
 //   warps 4..7   scale warps, one per TMEM lane quarter (SCALE_SETS sets of
 //                four can take turns by stage). Each lane reads the stage's X
 //                scale words from shared memory and the W scale words of its
@@ -36,14 +35,17 @@
 //                32q + l in column q of a 4-column group). One scale slot per
 //                shared-memory stage: the producer only loads a stage once the
 //                MMAs of the stage that last used its slot are done, so the
-//                one wait for the stage's bytes also frees the slot (and, in
-//                the first CTA, vouches for the operands); one arrival per
-//                stage on the first CTA's sf_full follows. Thread stores keep
-//                the in-order tensor pipe for MMAs only.
+//                one wait for the stage's X scales also frees the slot. The
+//                scale warps do not wait for the operands: each arrives once
+//                per stage on the first CTA's `full`, the barrier the TMA
+//                operand bytes complete on, so the MMA thread has a single
+//                wait per stage and the scale writes run while the operands
+//                are in flight. Thread stores keep the in-order tensor pipe
+//                for MMAs only.
 //   warp 1       first CTA only: the MMA issuer (one thread), eight
 //                block-scaled MMAs per stage (kind::mxf4nvf4 block16 for
 //                NVFP4, kind::mxf8f6f4 with E8M0 scales for MXFP8) after one
-//                wait on sf_full; one commit multicast to both CTAs' `empty`
+//                wait on `full`; one commit multicast to both CTAs' `empty`
 //                barriers per stage and, after a tile's last stage, to both
 //                `acc_full` barriers.
 //   warps 8..19  epilogue: three warps per lane quarter, at most two
@@ -80,6 +82,7 @@
 #include "common.cuh"
 #include "quant.cuh"
 
+#include <atomic>
 #include <mutex>
 
 namespace nvfp4moe {
@@ -104,6 +107,8 @@ constexpr int SFX_CHUNKS = 8, SFX_STAGE = 2 * SFX_CHUNKS * 512;
 // (640 x 96 = 61440); setmaxnreg moves some from warpgroup 0 to the
 // epilogue within that budget.
 constexpr int SCALE_SETS = 1;
+// the MMA thread waits on full[i % STAGES]: one scale-warp set
+static_assert(SCALE_SETS == 1, "the scale warps arrive on the MMA thread's `full` barrier");
 constexpr int SCALE_WARP0 = 4, EPI_WARP0 = SCALE_WARP0 + 4 * SCALE_SETS;
 constexpr int EPI_PER_QUARTER = 3, EPI_WARPS = 4 * EPI_PER_QUARTER;
 constexpr int NUM_THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
@@ -120,29 +125,34 @@ constexpr uint32_t TMEM_COLS = 512, TMEM_SF = MAX_N, SF_KB_COLS = 48, SF_SLOT_CO
 constexpr int OFF_W = 0;
 constexpr int OFF_X = OFF_W + STAGES * W_STAGE;
 constexpr int OFF_SFX = OFF_X + STAGES * X_STAGE;
-// barriers: full[SETS S], empty[S], sf_full[S], sf_loaded[SETS S], acc_full,
-// acc_empty. `full` and `sf_loaded` are waited on by the scale-warp set that
-// handles the stage: stage i uses barrier stage_bar(i) = (i % SETS) S +
+// barriers: full[SETS S], empty[S], sf_loaded[SETS S], acc_full, acc_empty.
+// `sf_loaded` is waited on by the scale-warp set that handles the stage: stage i uses barrier stage_bar(i) = (i % SETS) S +
 // (i / SETS) % S, so every barrier is waited on by one set, in order, and a
 // parity wait can never alias a phase two uses ahead.
 constexpr int OFF_BAR = OFF_SFX + STAGES * SFX_STAGE;
-constexpr int NUM_BARS = (2 * SCALE_SETS + 2) * STAGES + 2;
-constexpr int OFF_MISC = OFF_BAR + 8 * NUM_BARS;               // tmem base, abort flag
+constexpr int NUM_BARS = (2 * SCALE_SETS + 1) * STAGES + 2;
+constexpr int OFF_MISC = (OFF_BAR + 8 * NUM_BARS + 15) & ~15;  // tmem base, abort flag
 constexpr int OFF_GTAB = OFF_MISC + 16;  // per-group tile table (int4), one sentinel
+static_assert(OFF_BAR % 8 == 0 && OFF_GTAB % 16 == 0, "barriers and the int4 tile table stay aligned");
 constexpr int SMEM_BYTES = OFF_GTAB + 16 * (MAX_GROUPS + 1);
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 static_assert(X_KBLK % 1024 == 0, "k-block areas stay 1024-byte aligned");
 static_assert(TMEM_SF + STAGES * SF_SLOT_COLS <= TMEM_COLS, "TMEM columns");
 
-constexpr uint32_t FULL_COUNT = 1;        // the first CTA's producer
-constexpr uint32_t SF_FULL_COUNT = 8;     // 4 scale warps x 2 CTAs
+// the first CTA's `full` completes when the operand bytes of both CTAs have
+// landed and the scale warps of both CTAs (4 each) have written the stage's
+// block scales into TMEM: the producer's arrival plus eight.
+constexpr uint32_t FULL_COUNT = 1 + 8;
 constexpr uint32_t ACC_EMPTY_COUNT = 2 * EPI_WARPS;  // every epilogue warp of both CTAs
 
 __host__ __device__ constexpr uint32_t stage_bar(uint32_t i) {
     return (i % SCALE_SETS) * STAGES + (i / SCALE_SETS) % STAGES;
 }
 __host__ __device__ constexpr uint32_t stage_par(uint32_t i) { return ((i / SCALE_SETS) / STAGES) & 1u; }
+
+// Test hook flags (nvfp4moe_debug_gemm): normal operation uses none.
+constexpr uint32_t GEMM_DEBUG_WITHHOLD_LOADS = 1;  // producers issue nothing
 
 struct Params {
     int kind, epi, group_axis;
@@ -161,6 +171,15 @@ struct Params {
     void *c;
     float *amax;
     int32_t *err;  // device error word
+    uint64_t wait_ns;  // limit of every bounded wait
+    uint32_t debug;    // GEMM_DEBUG_* (test hook; 0 in normal operation)
+    // fused requantization of h (SwiGLU, NVFP4): hq == nullptr switches it off
+    uint8_t *hq, *hq_sc;
+    float *h_ts;
+    int32_t *rq_tiles;   // per group: epilogue-warp arrivals so far
+    int32_t *rq_cursor;  // per group: rows handed out so far
+    int32_t *rq_queue;   // published groups in order, g + 1 (0: slot not written yet)
+    int32_t *rq_ctr;     // [0] queue slots reserved, [1] head of the queue
 };
 
 struct Tile {
@@ -233,16 +252,16 @@ __device__ __forceinline__ Tile cursor_tile(const Params &p, const Cursor &c) {
     return T;
 }
 
-// Bounded wait that also gives up when another role of this CTA raised the
-// abort flag.
+// Bounded wait (limit_ns) that also gives up when another role of this CTA
+// raised the abort flag.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *abort_flag,
-                                              int32_t *err, int32_t id) {
+                                              int32_t *err, int32_t id, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > 2000000000ull) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             atomicCAS(err, 0, id);
             *abort_flag = 1;
             return false;
@@ -262,6 +281,134 @@ __device__ __forceinline__ uint32_t idesc_mxf8(int n, uint32_t sf_id) {
     return ((uint32_t)(n >> 3) << 17) | (1u << 23) | (16u << 24) | (sf_id << 29) | (sf_id << 4);
 }
 
+// ---------------------------------------------------------------------------
+// Fused requantization of h (the first GEMM of the expert FFN, NVFP4; the
+// entry point moe_expert_fwd_fused_requant).
+// An expert's NVFP4 tensor scale is amax(h) over all of its rows, known only
+// once the last of its tiles is stored. Every epilogue warp counts its tiles
+// per expert: one atomic per warp and tile, preceded by a fence that
+// publishes its h stores and its amax update, and deferred until the warp
+// has released the next accumulator, so that the stores have long drained.
+// The warp that makes the expert's last arrival publishes it: the decode
+// scale h_ts, then the expert's id in the next slot of a queue of experts.
+// When all epilogue warps of a CTA are done with their tiles they meet at a
+// CTA-local barrier and take rows from the queue until its head slot is not
+// written yet or everything is taken: rows are handed out by a fetch-and-add
+// on the head expert's row cursor (it never fails, so takers do not
+// serialize); the head moves on, with one compare-and-swap, only when its
+// expert has no rows left. Nothing ever waits on another CTA: every row still
+// gets requantized, because the warp that writes a queue slot is inside its
+// epilogue and drains the queue after it.
+// Measured on B200, this is slower than the standalone requantization after
+// GEMM1 (moe_expert_fwd): taking rows while tiles are still in flight, from
+// the epilogue or from otherwise idle warps, lengthens the GEMM's TMA
+// latency-bound pipeline by more than the separate pass costs.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int32_t ld_volatile_i32(const int32_t *p) {
+    return *reinterpret_cast<const volatile int32_t *>(p);
+}
+
+// Called by a whole warp after it stored its part of a tile of group g.
+__device__ __forceinline__ void requant_arrive(const Params &p, const int4 *gtab, int g, int lane) {
+    __threadfence();  // this lane's h stores (and lane 0's amax update) before the count
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(p.rq_tiles + g, 1) == gtab[g].x * (2 * EPI_WARPS) - 1;
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (!last) return;
+    if (lane == 0) {
+        __threadfence();  // every other warp's h and amax of g, seen through the count
+        p.h_ts[g] = nvfp4_ts(*reinterpret_cast<const volatile float *>(p.amax + g));
+        __threadfence();  // h_ts before the queue slot
+        const int32_t slot = atomicAdd(p.rq_ctr, 1);
+        *reinterpret_cast<volatile int32_t *>(p.rq_queue + slot) = g + 1;
+    }
+    __syncwarp();
+}
+
+// Takes up to max_rows rows of the expert at the head of the queue and
+// requantizes them (codes and MMA-layout scale words, as the standalone
+// grouped requantization writes them). Returns false, the same in every
+// lane, when the head slot is not written yet or the queue is used up. A slot
+// holding an impossible group is recorded (DEVERR_REQUANT) and passed over.
+__device__ __forceinline__ bool requant_take(const Params &p, const int4 *gtab, int G, int lane,
+                                             int max_rows, int &cg) {
+    int g = -1;
+    int32_t r = 0;
+    if (lane == 0) {
+        // the expert this warp took rows of last time: one fetch-and-add
+        if (cg >= 0) {
+            const int32_t got = atomicAdd(p.rq_cursor + cg, max_rows);
+            if (got < gtab[cg].w) {
+                g = cg;
+                r = got;
+            }
+        }
+        // else the head of the queue. Finite: every pass either hands out
+        // rows, stops, or finds the head moved past an exhausted expert (by
+        // this warp's CAS or another's)
+        while (g < 0) {
+            const int32_t s = ld_volatile_i32(p.rq_ctr + 1);
+            if (s >= G) break;
+            const int32_t e1 = ld_volatile_i32(p.rq_queue + s);
+            if (e1 == 0) break;
+            if (e1 < 1 || e1 > G) {
+                atomicCAS(p.err, 0, DEVERR_REQUANT);
+                atomicCAS(p.rq_ctr + 1, s, s + 1);
+                continue;
+            }
+            const int32_t got = atomicAdd(p.rq_cursor + (e1 - 1), max_rows);
+            if (got < gtab[e1 - 1].w) {
+                g = e1 - 1;
+                r = got;
+                break;
+            }
+            atomicCAS(p.rq_ctr + 1, s, s + 1);
+        }
+        cg = g;
+    }
+    g = __shfl_sync(0xFFFFFFFFu, g, 0);
+    if (g < 0) return false;
+    r = __shfl_sync(0xFFFFFFFFu, r, 0);
+    const int32_t row0 = gtab[g].y + r;
+    const int n = min(max_rows, gtab[g].w - r);
+    __threadfence();  // the slot was written after the group's amax was final
+    const float S_enc = nvfp4_senc(*reinterpret_cast<const volatile float *>(p.amax + g));
+    const int64_t f = p.f_out;
+    const int32_t G64 = (int32_t)(f / 64);
+    const uint16_t *h = static_cast<const uint16_t *>(p.c);
+    for (int32_t it = lane; it < n * G64; it += 32) {
+        const int64_t rr = row0 + it / G64;
+        const int32_t gr = it % G64;
+        const uint4 *pv = reinterpret_cast<const uint4 *>(h + rr * f + (int64_t)gr * 64);
+        uint4 raw[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) raw[j] = __ldcg(pv + j);
+        uint32_t scw = 0, w[8];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            float v[16];
+            unpack_bf16x8(raw[2 * b], v);
+            unpack_bf16x8(raw[2 * b + 1], v + 8);
+            scw |= nvfp4_block16(v, S_enc, w[2 * b], w[2 * b + 1]) << (8 * b);
+        }
+        uint4 *co = reinterpret_cast<uint4 *>(p.hq + rr * (f / 2) + (int64_t)gr * 32);
+        co[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        co[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        *reinterpret_cast<uint32_t *>(p.hq_sc + mma_sf_offset(rr, (int64_t)gr * 4, f / 16)) = scw;
+    }
+    __syncwarp();
+    return true;
+}
+
+// Epilogue warps only: CTA-local barrier (named barrier 1) of the 12
+// epilogue warps, all of which reach it after their tile loop (the warp is
+// reconverged first; the barrier itself is the non-aligned form).
+__device__ __forceinline__ void epilogue_barrier() {
+    __syncwarp();
+    asm volatile("barrier.sync 1, %0;" ::"n"(32 * EPI_WARPS) : "memory");
+}
+
 __device__ __forceinline__ float swiglu_value(float g, float u, float alpha) {
     const float gq = __fmul_rn(g, alpha);
     const float uq = __fmul_rn(u, alpha);
@@ -278,8 +425,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *empty = full + SCALE_SETS * STAGES;
-    uint64_t *sf_full = empty + STAGES;
-    uint64_t *sf_loaded = sf_full + STAGES;
+    uint64_t *sf_loaded = empty + STAGES;
     uint64_t *acc_full = sf_loaded + SCALE_SETS * STAGES;
     uint64_t *acc_empty = acc_full + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
@@ -308,6 +454,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         gtab[g] = e;
     }
     if (threadIdx.x == 0) *abort_flag = 0;
+    const bool requant = p.hq != nullptr;
+    // groups without rows are never published: their decode scale is 1
+    if (requant && blockIdx.x == 0)
+        for (int g = threadIdx.x; g < G; g += NUM_THREADS)
+            if (gtab[g].x == 0) p.h_ts[g] = 1.0f;
     __syncthreads();
     if (warp == 1) {
         tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -316,7 +467,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&empty[s], 1);
-            mbar_init(&sf_full[s], SF_FULL_COUNT);
         }
         for (int s = 0; s < SCALE_SETS * STAGES; ++s) {
             mbar_init(&full[s], FULL_COUNT);
@@ -345,7 +495,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const uint32_t sfc = nvf4 ? 4 : 1;  // scale chunks per k-block
             int s = 0;
             uint32_t phase = 0, i = 0;
-            bool ok = true;
+            // test hook: withhold every load (nothing is ever in flight), so
+            // that the consumers' bounded waits run out
+            bool ok = (p.debug & GEMM_DEBUG_WITHHOLD_LOADS) == 0;
             for (Cursor c = cursor_first(gtab, G, (int32_t)pair); c.g < G && ok && !*abort_flag;
                  cursor_next(gtab, G, npairs32, c)) {
                 const Tile T = cursor_tile(p, c);
@@ -359,22 +511,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int xcr = (int)((T.x_row + T.n - 1) / 128 - xa) + 1;
                 for (int kb0 = 0; kb0 < T.kt; kb0 += 2) {
                     const int nkb = T.kt - kb0 >= 2 ? 2 : 1;
-                    if (!wait_or_abort(&empty[s], phase ^ 1u, abort_flag, p.err, WAIT_GEMM_EMPTY)) {
+                    if (!wait_or_abort(&empty[s], phase ^ 1u, abort_flag, p.err, WAIT_GEMM_EMPTY, p.wait_ns)) {
                         ok = false;
                         break;
                     }
+                    // the X block scales first, on this CTA's own sf_loaded:
+                    // the scale warps start on them while the operands are
+                    // still in flight
                     const uint32_t sf_bytes = (uint32_t)xcr * nkb * sfc * 512u;
                     const uint32_t sb = stage_bar(i);
-                    uint64_t *sfbar = rank == 0 ? &full[sb] : &sf_loaded[sb];
-                    if (rank == 0)
-                        mbar_arrive_expect_tx(&full[sb], (uint32_t)nkb * kblk_tx + sf_bytes);
-                    else
-                        mbar_arrive_expect_tx(&sf_loaded[sb], sf_bytes);
+                    mbar_arrive_expect_tx(&sf_loaded[sb], sf_bytes);
                     const int64_t kc0 = nvf4 ? (int64_t)kb0 * 4 : (T.k0 / 128 + kb0);
                     uint8_t *ssf = smem + OFF_SFX + s * SFX_STAGE;
                     for (int cr = 0; cr < xcr; ++cr)
                         bulk_load(ssf + cr * (SFX_CHUNKS * 512), p.x_sc + ((xa + cr) * p.x_nkc + kc0) * 512,
-                                  nkb * sfc * 512u, sfbar);
+                                  nkb * sfc * 512u, &sf_loaded[sb]);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[sb], (uint32_t)nkb * kblk_tx);
                     const uint32_t cbar = cfull + 8u * sb;
                     for (int j = 0; j < nkb; ++j) {
                         const int32_t kx = (int32_t)(T.k0 + (int64_t)(kb0 + j) * 128);  // byte column
@@ -407,7 +559,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int w_rib = swiglu ? 64 * (int)rank + 16 * q + (lane & 15) : 32 * q + lane;
         const int64_t w_up = (swiglu && lane >= 16) ? p.f_out : 0;
         const uint32_t w_word = (uint32_t)((w_rib & 31) * 16 + (w_rib >> 5) * 4);
-        const uint32_t csf_full = cluster_addr(sf_full, 0);
+        const uint32_t c_full = cluster_addr(full, 0);
         const int chunks = nvf4 ? 4 : 1;  // scale chunks per k-block
 
         // a pipeline stage: tile at cursor c (T), k-blocks kb0 and kb0 + 1
@@ -449,12 +601,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         auto put = [&](const Stage &st, uint32_t i, const uint32_t (&w)[2][4]) -> bool {
             const Tile &T = st.T;
             const uint32_t s = i % STAGES, sb = stage_bar(i), par = stage_par(i);
-            // the stage's bytes landed (first CTA: operands and X scales on
-            // `full`; other CTA: its X scales on `sf_loaded`); the producer
-            // only loaded them after the MMAs that last read slot s were done
-            const bool ok = rank == 0 ? wait_or_abort(&full[sb], par, abort_flag, p.err, WAIT_GEMM_FULL)
-                                      : wait_or_abort(&sf_loaded[sb], par, abort_flag, p.err, WAIT_GEMM_SF_SLOT);
-            if (!ok) return false;
+            // the stage's X scales landed; the producer only loaded them
+            // after the MMAs that last read slot s were done, so the slot is
+            // free. The operands may still be in flight.
+            if (!wait_or_abort(&sf_loaded[sb], par, abort_flag, p.err, WAIT_GEMM_SF_SLOT, p.wait_ns)) return false;
             tc_fence_after();
             const int nkb = T.kt - st.kb0 >= 2 ? 2 : 1;
             // tile rows start at 128 a + 64 h: column j holds word (2h + j) % 4
@@ -496,8 +646,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if (rank == 0) mbar_arrive(&sf_full[s]);
-                else mbar_arrive_cluster_relaxed(csf_full + 8u * s);
+                if (rank == 0) mbar_arrive(&full[sb]);
+                else mbar_arrive_cluster_relaxed(c_full + 8u * sb);
             }
             return true;
         };
@@ -553,14 +703,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                  cursor_next(gtab, G, npairs32, c)) {
                 const Tile T = cursor_tile(p, c);
                 if (T.kt == 0) continue;
-                if (!wait_or_abort(acc_empty, acc_phase ^ 1u, abort_flag, p.err, WAIT_GEMM_ACC_EMPTY)) break;
+                if (!wait_or_abort(acc_empty, acc_phase ^ 1u, abort_flag, p.err, WAIT_GEMM_ACC_EMPTY, p.wait_ns)) break;
                 tc_fence_after();
                 const uint32_t idesc4 = idesc_nvf4(T.n);
                 for (int kb0 = 0; kb0 < T.kt; kb0 += 2) {
                     const int nkb = T.kt - kb0 >= 2 ? 2 : 1;
-                    // the scale warps arrive once the stage's scales are in
-                    // TMEM and (first CTA) its operands in shared memory
-                    if (!wait_or_abort(&sf_full[s], phase, abort_flag, p.err, WAIT_GEMM_SF_FULL)) {
+                    // one wait: both CTAs' operands landed and both CTAs'
+                    // scale warps wrote the stage's scales into TMEM
+                    if (!wait_or_abort(&full[s], phase, abort_flag, p.err, WAIT_GEMM_FULL, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -604,6 +754,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const bool up_lane = lane >= 16;
         const bool f32_out = p.epi == EPI_STORE_F32;
         uint32_t acc_phase = 0;
+        // fused requantization state: the group whose tile this warp stored
+        // last and has not counted yet (its count, with the fence before it,
+        // waits until the next tile so the stores have long drained), and the
+        // expert this warp takes rows of (lane 0)
+        int pend_g = -1, take_g = -1;
         for (Cursor c = cursor_first(gtab, G, (int32_t)pair); c.g < G && !*abort_flag;
              cursor_next(gtab, G, npairs32, c)) {
             const Tile T = cursor_tile(p, c);
@@ -616,7 +771,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int nb = max(0, min(2, T.n / 32 - b0));
             const int64_t row0 = T.out_row + 32 * b0;  // output row of the first column
             if (have_acc) {
-                if (!wait_or_abort(acc_full, acc_phase, abort_flag, p.err, WAIT_GEMM_ACC_FULL)) break;
+                if (!wait_or_abort(acc_full, acc_phase, abort_flag, p.err, WAIT_GEMM_ACC_FULL, p.wait_ns)) break;
                 tc_fence_after();
             }
             uint32_t va[32], vb[32];
@@ -634,6 +789,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster_relaxed(c_acc_empty);
                 acc_phase ^= 1u;
+            }
+            if (requant && pend_g >= 0) {
+                requant_arrive(p, gtab, pend_g, lane);
+                pend_g = -1;
             }
             float amax = 0.0f;
             // finish and store block b (0 or 1 of this warp) from its 32
@@ -693,6 +852,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (swiglu) {
                 amax = warp_max(amax);
                 if (lane == 0 && nb > 0) atomic_max_nonneg(p.amax + T.g, amax);
+                if (requant) pend_g = T.g;
+            }
+        }
+        if (requant) {
+            if (pend_g >= 0) requant_arrive(p, gtab, pend_g, lane);
+            // every epilogue warp of this CTA is past its tiles: take rows
+            // until the head of the queue is not written yet or all is taken
+            epilogue_barrier();
+            while (requant_take(p, gtab, G, lane, 4, take_g)) {
             }
         }
     } else {
@@ -807,6 +975,15 @@ cudaError_t launch_setup(int &grid) {
 
 }  // namespace
 
+// Test hook state, set by nvfp4moe_debug_gemm (abi.cu).
+std::atomic<uint32_t> g_gemm_debug{0};
+std::atomic<uint64_t> g_gemm_debug_wait_ns{2000000000ull};
+
+void set_gemm_debug(uint32_t flags, uint64_t wait_ns) {
+    g_gemm_debug_wait_ns.store(wait_ns ? wait_ns : 2000000000ull);
+    g_gemm_debug.store(flags);
+}
+
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     const bool nvf4 = a.kind == 0;
     const bool swiglu = a.epi == EPI_SWIGLU_AMAX;
@@ -834,7 +1011,21 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     p.wtiles = (int32_t)(swiglu ? p.f_out / 128 : a.N / 256);
     p.c = a.c;
     p.amax = a.amax;
+    if (a.hq) {
+        if (!swiglu || !nvf4 || !a.hq_sc || !a.h_ts || !a.rq_ws) return cudaErrorInvalidValue;
+        p.hq = a.hq;
+        p.hq_sc = a.hq_sc;
+        p.h_ts = a.h_ts;
+        int32_t *w = static_cast<int32_t *>(a.rq_ws);
+        const int64_t per = (a.G + 3) / 4 * 4;  // int32 arrays padded to 16 bytes
+        p.rq_tiles = w;
+        p.rq_cursor = w + per;
+        p.rq_queue = w + 2 * per;
+        p.rq_ctr = w + 3 * per;
+    }
     p.err = device_error_word();
+    p.debug = g_gemm_debug.load();
+    p.wait_ns = p.debug ? g_gemm_debug_wait_ns.load() : 2000000000ull;
     if (!p.err) return cudaErrorInvalidSymbol;
     // contraction bytes per row and scale chunks per 128-row block
     const int64_t kbytes = nvf4 ? a.a_cols / 2 : a.a_cols;

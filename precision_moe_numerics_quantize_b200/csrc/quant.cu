@@ -14,17 +14,12 @@ namespace nvfp4moe {
 
 __device__ int32_t g_device_error = 0;
 
+// Device address of g_device_error in the current device and context.
 int32_t *device_error_word() {
-    constexpr int kMaxDevices = 64;
-    static int32_t *addr[kMaxDevices] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<int32_t *>(p);
-    }
-    return addr[dev];
+    static SymbolAddressCache cache;
+    void *p = nullptr;
+    if (cached_symbol_address(cache, &g_device_error, &p) != cudaSuccess) return nullptr;
+    return static_cast<int32_t *>(p);
 }
 
 // ---------------------------------------------------------------------------
@@ -301,6 +296,133 @@ __global__ void __launch_bounds__(256, 3) mxfp8_cols_kernel(
         *reinterpret_cast<uint2 *>(codes + (c + 1) * rows + r0) = make_uint2(w1[0], w1[1]);
         *reinterpret_cast<uint2 *>(codes + (c + 2) * rows + r0) = make_uint2(w2[0], w2[1]);
         *reinterpret_cast<uint2 *>(codes + (c + 3) * rows + r0) = make_uint2(w3[0], w3[1]);
+        if (rq == 0) {
+            const int ks[4] = {k0, k1, k2, k3};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint8_t e8 = (uint8_t)(ks[j] + 127);
+                if (layout == NVFP4MOE_LAYOUT_ROWMAJOR)
+                    scales[(c + j) * G + b] = e8;
+                else
+                    scales[mma_sf_offset(c + j, b, G)] = e8;
+            }
+        }
+    }
+}
+
+// Column-wise MXFP8 over segments of rows: segment s holds rows
+// [seg_off[s], seg_off[s+1]) and is cut into ceil(len / 32) blocks of 32 rows,
+// the last one zero-padded. The blocks of all segments are packed in order
+// into an output of `pitch` columns (>= the packed total, a multiple of 32);
+// output columns past the packed blocks get zero codes and zero scale codes.
+// Each CTA first turns the segment lengths into block offsets in shared
+// memory; each warp then quantizes one 32-row block x 32-column patch, the
+// loads of rows outside the block's segment replaced by zeros. The draws
+// follow every element's row-major index in the [rows x cols] source.
+constexpr int MAX_SEGS = 1024;
+
+template <bool SR>
+__global__ void __launch_bounds__(256) mxfp8_cols_seg_kernel(
+    const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    const int32_t *__restrict__ seg_off, int32_t nseg, int64_t pitch, uint64_t seed,
+    uint64_t offset, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int layout) {
+    __shared__ int32_t blk0[MAX_SEGS + 1];  // first output block of each segment
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        // offsets must be non-decreasing inside [0, rows]; otherwise every
+        // output block is written as zeros, nothing is loaded, and the
+        // device error word records it
+        bool bad = lane == 0 && (seg_off[0] < 0 || seg_off[nseg] > rows);
+        int32_t run = 0;
+        for (int32_t base = 0; base < nseg; base += 32) {
+            const int32_t sidx = base + lane;
+            int32_t nb = 0;
+            if (sidx < nseg) {
+                const int32_t len = seg_off[sidx + 1] - seg_off[sidx];
+                bad |= len < 0;
+                nb = (len + 31) / 32;
+            }
+            int32_t incl = nb;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (sidx < nseg) blk0[sidx] = run + incl - nb;
+            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (__any_sync(0xFFFFFFFFu, bad)) {
+            run = 0;
+            if (lane == 0 && blockIdx.x == 0) atomicCAS(&g_device_error, 0, DEVERR_SEGMENTS);
+        }
+        if (lane == 0) blk0[nseg] = run;
+    }
+    __syncthreads();
+    const int32_t nblk = blk0[nseg];
+    const int rq = lane >> 3, cq = lane & 7;
+    const int64_t G = pitch / 32;   // scales per output row
+    const int64_t CP = cols / 32;   // column patches
+    const int64_t items = G * CP;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t it = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp; it < items; it += warps) {
+        const int64_t b = it / CP, cp = it - b * CP;
+        const int64_t c = cp * 32 + cq * 4;
+        int64_t r0 = 0, r_end = 0;  // source rows of this lane's 8 rows, segment end
+        if (b < nblk) {
+            int lo = 0, hi = nseg - 1;  // last segment whose first block <= b
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (blk0[mid] <= b) lo = mid; else hi = mid - 1;
+            }
+            r0 = (int64_t)seg_off[lo] + (b - blk0[lo]) * 32 + rq * 8;
+            r_end = seg_off[lo + 1];
+        }
+        uint2 q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            q[i] = (r0 + i < r_end) ? __ldg(reinterpret_cast<const uint2 *>(x + (r0 + i) * ld + c))
+                                    : make_uint2(0u, 0u);
+        float am0 = 0.0f, am1 = 0.0f, am2 = 0.0f, am3 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            am0 = fmaxf(am0, fabsf(bf16_lo(q[i].x)));
+            am1 = fmaxf(am1, fabsf(bf16_hi(q[i].x)));
+            am2 = fmaxf(am2, fabsf(bf16_lo(q[i].y)));
+            am3 = fmaxf(am3, fabsf(bf16_hi(q[i].y)));
+        }
+#pragma unroll
+        for (int m = 8; m <= 16; m <<= 1) {
+            am0 = fmaxf(am0, __shfl_xor_sync(0xFFFFFFFFu, am0, m));
+            am1 = fmaxf(am1, __shfl_xor_sync(0xFFFFFFFFu, am1, m));
+            am2 = fmaxf(am2, __shfl_xor_sync(0xFFFFFFFFu, am2, m));
+            am3 = fmaxf(am3, __shfl_xor_sync(0xFFFFFFFFu, am3, m));
+        }
+        const int k0 = mx_scale_exp(am0), k1 = mx_scale_exp(am1), k2 = mx_scale_exp(am2),
+                  k3 = mx_scale_exp(am3);
+        uint32_t w0[2] = {0u, 0u}, w1[2] = {0u, 0u}, w2[2] = {0u, 0u}, w3[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float v0 = scale_pow2(bf16_lo(q[i].x), k0), v1 = scale_pow2(bf16_hi(q[i].x), k1);
+            float v2 = scale_pow2(bf16_lo(q[i].y), k2), v3 = scale_pow2(bf16_hi(q[i].y), k3);
+            if (SR && r0 + i < r_end) {
+                const u32x4 r4 = philox_block(seed, offset, (uint64_t)((r0 + i) * cols + c) >> 2);
+                v0 = e4m3_sr_value(v0, r4.x);
+                v1 = e4m3_sr_value(v1, r4.y);
+                v2 = e4m3_sr_value(v2, r4.z);
+                v3 = e4m3_sr_value(v3, r4.w);
+            }
+            const uint32_t p01 = e4m3x2_hw(v0, v1), p23 = e4m3x2_hw(v2, v3);
+            const int h = i >> 2, sh = 8 * (i & 3);
+            w0[h] |= (p01 & 0xFFu) << sh;
+            w1[h] |= (p01 >> 8) << sh;
+            w2[h] |= (p23 & 0xFFu) << sh;
+            w3[h] |= (p23 >> 8) << sh;
+        }
+        const int64_t o = b * 32 + rq * 8;  // output column of this lane's first row
+        *reinterpret_cast<uint2 *>(codes + (c + 0) * pitch + o) = make_uint2(w0[0], w0[1]);
+        *reinterpret_cast<uint2 *>(codes + (c + 1) * pitch + o) = make_uint2(w1[0], w1[1]);
+        *reinterpret_cast<uint2 *>(codes + (c + 2) * pitch + o) = make_uint2(w2[0], w2[1]);
+        *reinterpret_cast<uint2 *>(codes + (c + 3) * pitch + o) = make_uint2(w3[0], w3[1]);
         if (rq == 0) {
             const int ks[4] = {k0, k1, k2, k3};
 #pragma unroll
@@ -615,6 +737,22 @@ cudaError_t launch_mxfp8_quantize(const uint16_t *x, int64_t rows, int64_t cols,
             mxfp8_cols_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seed, offset, codes,
                                                        scales, layout);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp8_quantize_seg(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                      const int32_t *seg_off, int32_t nseg, int64_t pitch,
+                                      uint64_t seed, uint64_t offset, int rounding,
+                                      uint8_t *codes, uint8_t *scales, int layout,
+                                      cudaStream_t s) {
+    if (pitch * cols == 0) return cudaSuccess;
+    const int g = grid_for((pitch / 32) * (cols / 32), 8);
+    if (rounding == NVFP4MOE_ROUND_SR)
+        mxfp8_cols_seg_kernel<true><<<g, 256, 0, s>>>(x, rows, cols, ld, seg_off, nseg, pitch, seed,
+                                                      offset, codes, scales, layout);
+    else
+        mxfp8_cols_seg_kernel<false><<<g, 256, 0, s>>>(x, rows, cols, ld, seg_off, nseg, pitch, seed,
+                                                       offset, codes, scales, layout);
     return cudaGetLastError();
 }
 

@@ -15,6 +15,12 @@ cudaError_t launch_nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols,
 cudaError_t launch_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts,
                                     int64_t rows, int64_t cols, int layout, float *out,
                                     cudaStream_t s);
+// Column-wise (axis 1) MXFP8 over segments of rows, blocks packed into an
+// output of `pitch` columns; see mxfp8_quantize_sr in nvfp4moe.h.
+cudaError_t launch_mxfp8_quantize_seg(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                      const int32_t *seg_off, int32_t nseg, int64_t pitch,
+                                      uint64_t seed, uint64_t offset, int rounding,
+                                      uint8_t *codes, uint8_t *scales, int layout, cudaStream_t s);
 cudaError_t launch_mxfp8_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                                   int axis, uint64_t seed, uint64_t offset, int rounding,
                                   uint8_t *codes, uint8_t *scales, int layout, cudaStream_t s);
@@ -71,8 +77,21 @@ struct GemmArgs {
     int64_t b_rows_per_group;  // rows of B per group (N, or 2f for SwiGLU)
     void *c;
     float *amax;      // SwiGLU: per-group amax of h
+    // SwiGLU with NVFP4: requantize h inside the same launch (hq != nullptr):
+    // hq [rows x f/2], hq_sc (MMA layout), h_ts [G]; rq_ws holds the expert
+    // queue, requant_ws_bytes(G) bytes, zeroed before the launch.
+    uint8_t *hq = nullptr, *hq_sc = nullptr;
+    float *h_ts = nullptr;
+    void *rq_ws = nullptr;
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s);
+// Workspace of the fused requantization: per-group arrival counters, row
+// cursors and queue slots (int32, each array padded to 16 bytes), then the
+// two queue counters.
+inline size_t requant_ws_bytes(int64_t G) { return (size_t)(3 * ((G + 3) / 4 * 4) + 4) * 4; }
+// Test hook of the failure path (nvfp4moe_debug_gemm).
+void set_gemm_debug(uint32_t flags, uint64_t wait_ns);
+
 // Device address of the device error word on the current device, for kernels
 // built as whole programs (they cannot name the variable itself); nullptr if
 // the runtime cannot resolve it.

@@ -396,35 +396,20 @@ static constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
 // Every GPU that loads the library keeps this array until the process exits.
 static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocScratchBytes];
 
-// Device address of g_route_scratch on the current device. In host code the
-// array's name is only a stand-in, so the address is looked up once per
-// device with cudaGetSymbolAddress (the first call on a device) and cached.
+// Device address of g_route_scratch in the current device and context. In
+// host code the array's name is only a stand-in, so the address is looked up
+// with cudaGetSymbolAddress on the first call in each device and driver
+// context (the module, and with it the array, is loaded once per context)
+// and cached.
 static void *route_scratch_address(nvfp4moe_status *st) {
-    constexpr int kMaxDevices = 64;
-    static std::mutex mu;
-    static void *addr[kMaxDevices] = {};
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SymbolAddressCache cache;
+    void *p = nullptr;
+    cudaError_t e = cached_symbol_address(cache, g_route_scratch, &p);
     if (e != cudaSuccess) {
-        *st = cuda_status(e, "moe_route_permute_noalloc: cudaGetDevice");
+        *st = cuda_status(e, "moe_route_permute_noalloc: cudaGetSymbolAddress");
         return nullptr;
     }
-    if (dev < 0 || dev >= kMaxDevices) {
-        set_last_error("moe_route_permute_noalloc: device %d out of range", dev);
-        *st = NVFP4MOE_ERR_INVALID_ARG;
-        return nullptr;
-    }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_route_scratch);
-        if (e != cudaSuccess) {
-            *st = cuda_status(e, "moe_route_permute_noalloc: cudaGetSymbolAddress");
-            return nullptr;
-        }
-        addr[dev] = p;
-    }
-    return addr[dev];
+    return p;
 }
 
 }  // namespace nvfp4moe

@@ -41,12 +41,15 @@ _SIGS = {
     "nvfp4moe_version": (C.c_int, []),
     "nvfp4moe_last_error": (C.c_char_p, []),
     "nvfp4moe_device_error": (C.c_int, [_P]),
+    "nvfp4moe_debug_gemm": (C.c_int, [C.c_uint32, _U64]),
     "nvfp4moe_max_rows": (_I64, [_I64, _I32, _I32]),
     "nvfp4moe_selftest": (C.c_int, [_I, _P, _P]),
     "nvfp4moe_amax_bf16": (C.c_int, [_P, _I64, _I64, _I64, _P, _P]),
     "nvfp4_quantize": (C.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P]),
     "nvfp4_dequantize": (C.c_int, [_P, _P, _P, _I64, _I64, _I, _P, _P]),
-    "mxfp8_quantize_sr": (C.c_int, [_P, _I64, _I64, _I64, _I, _U64, _U64, _I, _P, _P, _I, _P]),
+    "mxfp8_quantize_sr": (C.c_int, [_P, _I64, _I64, _I64, _I, _P, _I32, _U64, _U64, _I, _P, _P, _I,
+                                    _P]),
+    "nvfp4moe_mxfp8_seg_rows": (C.c_int64, [_I64, _I32]),
     "mxfp8_dequantize": (C.c_int, [_P, _P, _I64, _I64, _I, _P, _P]),
     "rht32_quantize": (C.c_int, [_P, _I64, _I64, _I64, _U64, _I, _P, _P, _P, _P, _I, _P]),
     "rht32_dequantize": (C.c_int, [_P, _P, _P, _I64, _I64, _U64, _I, _I, _P, _P]),
@@ -57,6 +60,10 @@ _SIGS = {
                                             _P, _P, _P, _P, _P, _P]),
     "moe_expert_fwd": (C.c_int, [_P, _P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                  _P, _P, _P, _P, _P, _I64, _P]),
+    "moe_expert_fwd_fused_requant_workspace_size": (_SZ, [_I32]),
+    "moe_expert_fwd_fused_requant": (C.c_int, [_P, _P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P,
+                                               _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _SZ,
+                                               _P]),
     "moe_expert_fwd_mxfp8": (C.c_int, [_P, _P, _P, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _I64, _P]),
     "swiglu_bwd": (C.c_int, [_P, _P, _I64, _I64, _P, _P]),
@@ -115,6 +122,14 @@ def version():
     return lib().nvfp4moe_version()
 
 
+def debug_gemm(flags, wait_ns=0):
+    """Test hook of the GEMMs' failure path (see include/nvfp4moe.h)."""
+    _check("nvfp4moe_debug_gemm", lib().nvfp4moe_debug_gemm(flags, wait_ns))
+
+
+DEBUG_WITHHOLD_LOADS = 1
+
+
 def device_error():
     code = C.c_int32(0)
     st = lib().nvfp4moe_device_error(C.byref(code))
@@ -152,11 +167,18 @@ def nvfp4_dequantize(codes, scales, ts, rows, cols, out, layout=LAYOUT_ROWMAJOR,
 
 
 def mxfp8_quantize_sr(x, codes, scales, axis=0, seed=0, offset=0, rounding=ROUND_SR,
-                      layout=LAYOUT_ROWMAJOR, ld=None, stream=None):
+                      layout=LAYOUT_ROWMAJOR, ld=None, seg_off=None, stream=None):
+    """seg_off: device int32 [nseg + 1] (axis 1 only); codes then have
+    mxfp8_seg_rows(rows, nseg) columns."""
     rows, cols = x.shape
+    nseg = 0 if seg_off is None else seg_off.numel() - 1
     _check("mxfp8_quantize_sr", lib().mxfp8_quantize_sr(
-        _ptr(x), rows, cols, ld or cols, axis, seed, offset, rounding, _ptr(codes), _ptr(scales),
-        layout, _stream(stream)))
+        _ptr(x), rows, cols, ld or cols, axis, _ptr(seg_off), nseg, seed, offset, rounding,
+        _ptr(codes), _ptr(scales), layout, _stream(stream)))
+
+
+def mxfp8_seg_rows(rows, nseg):
+    return lib().nvfp4moe_mxfp8_seg_rows(rows, nseg)
 
 
 def mxfp8_dequantize(codes, scales, out, layout=LAYOUT_ROWMAJOR, stream=None):
@@ -210,6 +232,22 @@ def moe_expert_fwd(xq, xq_sc, x_ts, expert_off, E, d, f, w1, w1_sc, w1_ts, w2, w
         _ptr(xq), _ptr(xq_sc), _ptr(x_ts), _ptr(expert_off), E, d, f, _ptr(w1), _ptr(w1_sc),
         _ptr(w1_ts), _ptr(w2), _ptr(w2_sc), _ptr(w2_ts), _ptr(h), _ptr(hq), _ptr(hq_sc),
         _ptr(h_amax), _ptr(h_ts), _ptr(y), rows_alloc, _stream(stream)))
+
+
+def moe_expert_fwd_fused_requant_workspace_size(E):
+    return lib().moe_expert_fwd_fused_requant_workspace_size(E)
+
+
+def moe_expert_fwd_fused_requant(xq, xq_sc, x_ts, expert_off, E, d, f, w1, w1_sc, w1_ts, w2,
+                                 w2_sc, w2_ts, h, hq, hq_sc, h_amax, h_ts, y, rows_alloc, ws,
+                                 stream=None):
+    """moe_expert_fwd with the requantization of h fused into GEMM1; ws: device
+    workspace of moe_expert_fwd_fused_requant_workspace_size(E) bytes."""
+    _check("moe_expert_fwd_fused_requant", lib().moe_expert_fwd_fused_requant(
+        _ptr(xq), _ptr(xq_sc), _ptr(x_ts), _ptr(expert_off), E, d, f, _ptr(w1), _ptr(w1_sc),
+        _ptr(w1_ts), _ptr(w2), _ptr(w2_sc), _ptr(w2_ts), _ptr(h), _ptr(hq), _ptr(hq_sc),
+        _ptr(h_amax), _ptr(h_ts), _ptr(y), rows_alloc, _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def moe_expert_fwd_mxfp8(xq, xq_sc, expert_off, E, d, f, w1, w1_sc, w2, w2_sc, h, h_amax, hq,

@@ -59,9 +59,14 @@ P = 1 << 20  # a fake, 16-byte aligned "device pointer"; validation fails before
     (lambda L: L.nvfp4_quantize(None, 4, 64, 64, None, P, P, P + 16, 0, None), 1),   # null
     (lambda L: L.nvfp4_quantize(P, 4, 64, 64, P + 16, P, P, P + 16, 0, None), 1),    # alias
     (lambda L: L.nvfp4_quantize(P, 4, 64, 64, None, P, P, P + 16, 7, None), 1),      # layout
-    (lambda L: L.mxfp8_quantize_sr(P, 4, 64, 64, 2, 0, 0, 1, P, P, 0, None), 1),     # axis
-    (lambda L: L.mxfp8_quantize_sr(P, 40, 64, 64, 1, 0, 0, 1, P, P, 0, None), 2),    # rows % 32
-    (lambda L: L.mxfp8_quantize_sr(P, 4, 64, 64, 0, 0, 0, 5, P, P, 0, None), 1),     # rounding
+    (lambda L: L.mxfp8_quantize_sr(P, 4, 64, 64, 2, None, 0, 0, 0, 1, P, P, 0, None), 1),  # axis
+    (lambda L: L.mxfp8_quantize_sr(P, 40, 64, 64, 1, None, 0, 0, 0, 1, P, P, 0, None), 2), # rows % 32
+    (lambda L: L.mxfp8_quantize_sr(P, 4, 64, 64, 0, None, 0, 0, 0, 5, P, P, 0, None), 1),  # rounding
+    (lambda L: L.mxfp8_quantize_sr(P, 40, 64, 64, 0, P, 2, 0, 0, 1, P, P, 0, None), 1),    # seg + axis 0
+    (lambda L: L.mxfp8_quantize_sr(P, 40, 64, 64, 1, P, 0, 0, 0, 1, P, P, 0, None), 1),    # nseg 0
+    (lambda L: L.mxfp8_quantize_sr(P, 40, 64, 64, 1, P, 1025, 0, 0, 1, P, P, 0, None), 1), # nseg > 1024
+    (lambda L: L.mxfp8_quantize_sr(P, 40, 96, 96, 1, P, 2, 0, 0, 1, P, P, 0, None), 2),    # cols % 64
+    (lambda L: L.mxfp8_quantize_sr(P, 40, 64, 64, 1, P + 2, 2, 0, 0, 1, P, P, 0, None), 3),  # seg_off align
     (lambda L: L.rht32_quantize(P, 4, 48, 48, 0, 0, None, P, P, P, 0, None), 2),     # cols % 32
     (lambda L: L.rht32_quantize(P, 4, 64, 64, 0, 0, None, P, P, P, 1, None), 7),     # MMA layout
     (lambda L: L.moe_route_permute(P, P, 8, 4, 5, 64, 1, None, P, P, P, P, P, P, P, P, P,
@@ -72,6 +77,8 @@ P = 1 << 20  # a fake, 16-byte aligned "device pointer"; validation fails before
                                    1 << 20, None), 2),                               # d % 64
     (lambda L: L.moe_expert_fwd(P, P, P, P, 4, 384, 256, P, P, P, P, P, P, P, P, P, P, P, P,
                                 128, None), 2),                                      # d % 256
+    (lambda L: L.moe_expert_fwd_fused_requant(P, P, P, P, 4, 256, 256, P, P, P, P, P, P, P, P,
+                                              P, P, P, P, 128, P, 16, None), 4),     # workspace
     (lambda L: L.moe_expert_fwd_mxfp8(P, P, P, 4, 384, 256, P, P, P, P, P, P, P, P, P, 128,
                                       None), 2),                                     # d % 256
     (lambda L: L.moe_expert_fwd_mxfp8(P, P, P, 4, 256, 256, P, P, P, P, P, P, P, P, P, 100,

@@ -101,7 +101,9 @@ def test_expert_bwd_gemm1_matches_oracle(dev, lib, orc):
         s = slice(off[e], off[e + 1])
         wc, ws = orc.mxfp8_quantize(synth.bf16_bits_to_f32(W1[e]), axis=1, rounding=0)
         mag = orc.gemm_f64(np.abs(Gd[s]), np.abs(orc.mxfp8_dequantize(wc, ws).astype(np.float64)))
-        assert np.all(np.abs(got_dx[s] - ref_dx[s]) <= 2 * _ulp(ref_dx[s]) + 1e-5 * mag + 1e-30), e
+        # one bf16 ulp (at the larger magnitude) on top of the accumulator bound
+        ulp = _ulp(np.maximum(np.abs(ref_dx[s]), np.abs(got_dx[s])))
+        assert np.all(np.abs(got_dx[s] - ref_dx[s]) <= ulp + 1e-5 * mag + 1e-30), e
         magw = orc.gemm_f64(np.abs(Td[:, s]), np.abs(Xd[:, s]))
         refw = ref["dw1"][e].astype(np.float64)
         assert np.all(np.abs(got_dw[e] - refw) <= 1e-5 * magw + 2.0 ** -23 * np.abs(refw) + 1e-30), e

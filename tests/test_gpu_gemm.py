@@ -216,3 +216,37 @@ def test_mxfp8_gemm_group_k(dev, lib, orc, M):
         sl = slice(off[g], off[g + 1])
         _check_f32(got[g], orc.gemm_f64(Ad[:, sl], Bd[:, sl]),
                    orc.gemm_f64(np.abs(Ad[:, sl]), np.abs(Bd[:, sl])))
+
+
+def test_bounded_wait_gives_up_and_the_context_survives(dev, lib, orc):
+    """The failure path of the GEMM pipeline, without a fault: with the test
+    hook set, the producers issue no load at all (nothing is in flight), so
+    the MMA thread's and the scale warps' bounded waits run out after 10 ms;
+    every role winds down, the launch ends, and the device error word holds
+    the id of the wait that gave up first (the MMA thread's wait on `full`
+    or a scale warp's wait on its scales). The same GEMM then runs normally
+    on the same context and matches the oracle."""
+    A = _f32(synth.rows_np(0, synth.TAG_A, 0, 128, 256, 1.0))
+    W = _f32(synth.rows_np(0, synth.TAG_W, 0, 256, 256, 0.02))
+    ac, as_, at = _quant(orc, A)
+    wc, ws, wt = _quant(orc, W)
+    args = [dev_u8(ac, dev), dev_u8(rowmajor_to_mma(as_), dev), dev_f32([at], dev), 0,
+            dev_u8(wc, dev), dev_u8(rowmajor_to_mma(ws), dev), dev_f32([wt], dev),
+            torch.tensor([0, 128], dtype=torch.int32, device=dev), 1, 128, 256, 256]
+    c = torch.zeros(128, 256, dtype=torch.float32, device=dev)
+    assert lib.device_error() == (0, 0)
+    lib.debug_gemm(lib.DEBUG_WITHHOLD_LOADS, 10_000_000)
+    try:
+        lib.nvfp4_grouped_gemm(*args, c, out_dtype=lib.OUT_F32)
+        sync()
+    finally:
+        lib.debug_gemm(0)
+    st, code = lib.device_error()
+    assert st == 6 and code in (1, 6), (st, code)  # NVFP4MOE_ERR_TIMEOUT; WAIT_GEMM_FULL / _SF_SLOT
+    assert lib.device_error() == (0, 0)  # read and cleared
+    lib.nvfp4_grouped_gemm(*args, c, out_dtype=lib.OUT_F32)
+    sync()
+    Ad = orc.nvfp4_to_f64(ac, as_, at, 128, 256)
+    Wd = orc.nvfp4_to_f64(wc, ws, wt, 256, 256)
+    _check_f32(c.cpu().numpy(), orc.gemm_f64(Ad, Wd), orc.gemm_f64(np.abs(Ad), np.abs(Wd)))
+    assert lib.device_error() == (0, 0)

@@ -8,9 +8,14 @@ oracle's own inputs:
   h    within one bf16 ulp plus the propagated accumulator tolerance
        (1e-5 * sum |a b| on g and u, through dh/dg and dh/du);
   h_amax equal to max |h| of the GPU's own h (the fused reduction);
-  hq   codes equal to the oracle's except where h itself differed (flip
-       fraction below 1e-3);
-  y    within one bf16 ulp plus 1e-5 * sum |a b| on rows whose hq agrees.
+  hq   every 16-element block whose h is bit-identical to the oracle's, in an
+       expert whose tensor scale matches, has the oracle's codes and scale;
+       codes differ from the oracle's in under 1e-3 of all positions;
+  y    within one bf16 ulp plus 1e-5 * sum |a b| on rows whose hq agrees; the
+       number of experts and rows this covers is asserted, not skipped.
+An fp32 accumulator rounded once to bf16 and an fp64 value rounded once to
+bf16 differ by at most one bf16 ulp (of the larger magnitude) plus the
+accumulator's own error, which is the bound used for h and y.
 """
 import numpy as np
 import pytest
@@ -139,9 +144,21 @@ def _ulp(v):
     return np.exp2(np.floor(np.log2(np.maximum(np.abs(v), 1e-38))) - 7)
 
 
+def _ulp2(a, b):
+    """One bf16 ulp at the larger of two magnitudes."""
+    return _ulp(np.maximum(np.abs(a), np.abs(b)))
+
+
+def _blocks_same(a, b, n, blk):
+    """Per (row, block of blk elements): all elements equal."""
+    return np.all((a == b).reshape(n, -1, blk), axis=2)
+
+
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("router", ["uniform", "zipf"])
-def test_expert_fwd_small_layer(dev, lib, orc, router):
-    """2048 tokens, d = 1024, f = 512, 32 experts, top-4."""
+def test_expert_fwd_small_layer(dev, lib, orc, router, fused):
+    """2048 tokens, d = 1024, f = 512, 32 experts, top-4; the default entry
+    point and the one with the requantization fused into GEMM1."""
     sh = synth.SHAPES["small_moe"]
     T, d, f, E, k = sh.T, sh.d, sh.f, sh.E, sh.k
     logits = (synth.logits_uniform_np(2, T, E) if router == "uniform"
@@ -156,17 +173,24 @@ def test_expert_fwd_small_layer(dev, lib, orc, router):
     xsc[real] = xs[tok[real]]
     w1c, w1s, w1t = _quant_experts(orc, 1, synth.TAG_W1, E, 2 * f, d)
     w2c, w2s, w2t = _quant_experts(orc, 1, synth.TAG_W2, E, d, f)
-    h = torch.empty(R, f, dtype=torch.bfloat16, device=dev)
+    # rows past the last expert are never written: zero-filled so that the
+    # host copies below convert cleanly
+    h = torch.zeros(R, f, dtype=torch.bfloat16, device=dev)
     hq = torch.empty(R, f // 2, dtype=torch.uint8, device=dev)
     hq_sc = torch.empty(R * f // 16, dtype=torch.uint8, device=dev)
     h_amax = torch.empty(E, device=dev)
     h_ts = torch.empty(E, device=dev)
-    y = torch.empty(R, d, dtype=torch.bfloat16, device=dev)
-    lib.moe_expert_fwd(dev_u8(xq, dev), dev_u8(rowmajor_to_mma(xsc), dev), dev_f32([xts], dev),
-                       torch.tensor(off, device=dev), E, d, f, dev_u8(w1c, dev),
-                       dev_u8(rowmajor_to_mma(w1s), dev), dev_f32(w1t, dev), dev_u8(w2c, dev),
-                       dev_u8(rowmajor_to_mma(w2s), dev), dev_f32(w2t, dev), h, hq, hq_sc, h_amax,
-                       h_ts, y, R)
+    y = torch.zeros(R, d, dtype=torch.bfloat16, device=dev)
+    args = [dev_u8(xq, dev), dev_u8(rowmajor_to_mma(xsc), dev), dev_f32([xts], dev),
+            torch.tensor(off, device=dev), E, d, f, dev_u8(w1c, dev),
+            dev_u8(rowmajor_to_mma(w1s), dev), dev_f32(w1t, dev), dev_u8(w2c, dev),
+            dev_u8(rowmajor_to_mma(w2s), dev), dev_f32(w2t, dev), h, hq, hq_sc, h_amax, h_ts, y, R]
+    if fused:
+        ws = torch.empty(lib.moe_expert_fwd_fused_requant_workspace_size(E), dtype=torch.uint8,
+                         device=dev)
+        lib.moe_expert_fwd_fused_requant(*args, ws)
+    else:
+        lib.moe_expert_fwd(*args)
     sync()
     gh = _f32(host_bits(h)).astype(np.float64)
     ghq = host_u8(hq)
@@ -174,7 +198,9 @@ def test_expert_fwd_small_layer(dev, lib, orc, router):
     gy = _f32(host_bits(y)).astype(np.float64)
     gam = h_amax.cpu().numpy()
     gts = h_ts.cpu().numpy()
+    ghb = host_bits(h)
     flips = total = 0
+    experts_used = experts_y = rows_used = rows_y = blocks = total_blocks = 0
     for e in range(E):
         rows = np.arange(off[e], off[e + 1])
         rows_real = rows[tok[rows] >= 0]
@@ -182,6 +208,9 @@ def test_expert_fwd_small_layer(dev, lib, orc, router):
             assert gam[e] == 0.0
             continue
         n = len(rows_real)
+        experts_used += 1
+        rows_used += n
+        assert np.isfinite(gh[rows_real]).all() and np.isfinite(gy[rows_real]).all(), e
         r = orc.expert_ffn(xq[rows_real], xsc[rows_real], xts, w1c[e * 2 * f:(e + 1) * 2 * f],
                            w1s[e * 2 * f:(e + 1) * 2 * f], w1t[e], w2c[e * d:(e + 1) * d],
                            w2s[e * d:(e + 1) * d], w2t[e])
@@ -196,27 +225,43 @@ def test_expert_fwd_small_layer(dev, lib, orc, router):
         dh_dg = np.abs((sig * (1 + g * (1 - sig))) * u)
         dh_du = np.abs(g * sig)
         href = _f32(r["h"]).astype(np.float64)
-        tol = _ulp(href) + dh_dg * mag[:, :f] + dh_du * mag[:, f:] + 1e-30
+        tol = _ulp2(href, gh[rows_real]) + dh_dg * mag[:, :f] + dh_du * mag[:, f:] + 1e-30
         assert np.all(np.abs(gh[rows_real] - href) <= tol), e
         # fused amax equals the max of the GPU's own h; padding rows are zero
         assert gam[e] == np.abs(gh[rows]).max()
         assert not gh[rows[tok[rows] < 0]].any()
         assert gts[e] == np.float32(np.float32(gam[e]) / np.float32(2688.0))
-        # requantized codes: flips only where h differed
-        same = np.all(ghq[rows_real] == r["hq"], axis=1) & np.all(ghs[rows_real] == r["hq_sc"],
-                                                                   axis=1)
         flips += int(np.sum(ghq[rows_real] != r["hq"]))
         total += r["hq"].size
+        if gts[e] != r["h_ts"]:
+            continue  # the expert's tensor scale moved: no code is comparable
+        # requantized codes: every 16-block whose h is bit-identical has the
+        # oracle's codes (8 bytes) and scale
+        hb_same = _blocks_same(ghb[rows_real], r["h"], n, 16)
+        codes_same = _blocks_same(ghq[rows_real], r["hq"], n, 8)
+        sc_same = ghs[rows_real] == r["hq_sc"]
+        assert np.all(codes_same[hb_same] & sc_same[hb_same]), e
+        blocks += int(hb_same.sum())
+        total_blocks += hb_same.size
         # y on rows whose hq agrees
+        same = np.all(ghq[rows_real] == r["hq"], axis=1) & np.all(ghs[rows_real] == r["hq_sc"],
+                                                                   axis=1)
         H = orc.nvfp4_to_f64(r["hq"], r["hq_sc"], r["h_ts"], n, f)
         W2 = orc.nvfp4_to_f64(w2c[e * d:(e + 1) * d], w2s[e * d:(e + 1) * d], w2t[e], d, f)
         ymag = orc.gemm_f64(np.abs(H), np.abs(W2)) * 1e-5
         yref = _f32(r["y"]).astype(np.float64)
-        if gts[e] == r["h_ts"]:
-            ok = np.abs(gy[rows_real] - yref) <= _ulp(yref) * 2 + ymag + 1e-30
-            assert np.all(ok[same]), e
+        ok = np.abs(gy[rows_real] - yref) <= _ulp2(yref, gy[rows_real]) + ymag + 1e-30
+        assert np.all(ok[same]), e
         assert not gy[rows[tok[rows] < 0]].any()
+        experts_y += 1
+        rows_y += int(same.sum())
     assert flips <= 1e-3 * total, (flips, total)
+    # h agrees bit for bit in almost every block, and y was compared on
+    # nearly every expert and row (a tensor-scale mismatch is rare: it needs
+    # the expert's largest |h| to be one of the values one ulp apart)
+    assert blocks >= 0.99 * total_blocks, (blocks, total_blocks)
+    assert experts_y >= 0.9 * experts_used, (experts_y, experts_used)
+    assert rows_y >= 0.9 * rows_used, (rows_y, rows_used)
 
 
 def _mx_experts(orc, seed, tag, E, rows, cols):
@@ -254,11 +299,11 @@ def test_expert_fwd_mxfp8_small_layer(dev, lib, orc, router):
     xsc[real] = xs_t[tok[real]]
     w1c, w1s = _mx_experts(orc, 1, synth.TAG_W1, E, 2 * f, d)
     w2c, w2s = _mx_experts(orc, 1, synth.TAG_W2, E, d, f)
-    h = torch.empty(R, f, dtype=torch.bfloat16, device=dev)
+    h = torch.zeros(R, f, dtype=torch.bfloat16, device=dev)
     h_amax = torch.empty(E, device=dev)
     hq = torch.empty(R, f, dtype=torch.uint8, device=dev)
     hq_sc = torch.empty(R * f // 32, dtype=torch.uint8, device=dev)
-    y = torch.empty(R, d, dtype=torch.bfloat16, device=dev)
+    y = torch.zeros(R, d, dtype=torch.bfloat16, device=dev)
     lib.moe_expert_fwd_mxfp8(dev_u8(xq, dev), dev_u8(rowmajor_to_mma(xsc), dev),
                              torch.tensor(off, device=dev), E, d, f, dev_u8(w1c, dev),
                              dev_u8(rowmajor_to_mma(w1s), dev), dev_u8(w2c, dev),
@@ -270,7 +315,7 @@ def test_expert_fwd_mxfp8_small_layer(dev, lib, orc, router):
     ghs = mma_to_rowmajor(host_u8(hq_sc), R, f // 32)
     gy = _f32(host_bits(y)).astype(np.float64)
     gam = h_amax.cpu().numpy()
-    blocks = total_blocks = 0
+    blocks = total_blocks = rows_y = rows_used = 0
     for e in range(E):
         rows = np.arange(off[e], off[e + 1])
         rows_real = rows[tok[rows] >= 0]
@@ -278,6 +323,7 @@ def test_expert_fwd_mxfp8_small_layer(dev, lib, orc, router):
             assert gam[e] == 0.0
             continue
         n = len(rows_real)
+        assert np.isfinite(gh[rows_real]).all() and np.isfinite(gy[rows_real]).all(), e
         W1 = slice(e * 2 * f, (e + 1) * 2 * f)
         W2 = slice(e * d, (e + 1) * d)
         r = orc.expert_ffn_mxfp8(xq[rows_real], xsc[rows_real], w1c[W1], w1s[W1], w2c[W2],
@@ -289,7 +335,7 @@ def test_expert_fwd_mxfp8_small_layer(dev, lib, orc, router):
         g, u = gu[:, :f], gu[:, f:]
         sig = 1.0 / (1.0 + np.exp(-g))
         href = _f32(r["h"]).astype(np.float64)
-        tol = (_ulp(href) + np.abs(sig * (1 + g * (1 - sig)) * u) * mag[:, :f]
+        tol = (_ulp2(href, gh[rows_real]) + np.abs(sig * (1 + g * (1 - sig)) * u) * mag[:, :f]
                + np.abs(g * sig) * mag[:, f:] + 1e-30)
         assert np.all(np.abs(gh[rows_real] - href) <= tol), e
         assert gam[e] == np.abs(gh[rows]).max()
@@ -308,8 +354,11 @@ def test_expert_fwd_mxfp8_small_layer(dev, lib, orc, router):
         B2 = _mx_f64(orc, w2c[W2], w2s[W2])
         ymag = orc.gemm_f64(np.abs(H), np.abs(B2)) * 1e-5
         yref = _f32(r["y"]).astype(np.float64)
-        ok = np.abs(gy[rows_real] - yref) <= _ulp(yref) * 2 + ymag + 1e-30
+        ok = np.abs(gy[rows_real] - yref) <= _ulp2(yref, gy[rows_real]) + ymag + 1e-30
         assert np.all(ok[same]), e
         assert not gy[rows[tok[rows] < 0]].any()
+        rows_y += int(same.sum())
+        rows_used += n
+    assert rows_y >= 0.9 * rows_used, (rows_y, rows_used)
     # h itself agrees bit for bit in almost every block
     assert blocks >= 0.99 * total_blocks, (blocks, total_blocks)

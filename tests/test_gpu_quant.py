@@ -197,3 +197,49 @@ def test_empty_inputs(dev, lib):
     lib.nvfp4_quantize(x, codes, codes, ts, rows=0, cols=64)
     sync()
     assert ts.item() == 1.0
+
+
+@pytest.mark.parametrize("rounding,layout", [(1, 0), (0, 0), (1, 1)])
+def test_mxfp8_cols_unaligned_segments(dev, lib, orc, rounding, layout):
+    """Column-wise MXFP8 over segments that do not start on 32-row boundaries
+    (one of them empty): each segment cut into 32-row blocks, the last one
+    zero-padded, blocks packed in order; bit-exact against the oracle, which
+    pads each segment the same way. Columns past the packed blocks are zero."""
+    rows, cols = 200, 128
+    seg = np.array([0, 20, 20, 75, 150, 200], np.int32)
+    bits = synth.grad_rows_np(9, 0, rows, cols, synth.outlier_channels(9, cols, 2))
+    x = _f32(bits)
+    rc, rs = orc.mxfp8_quantize(x, axis=1, seg_off=seg, seed=7, offset=1, rounding=rounding)
+    P = lib.mxfp8_seg_rows(rows, len(seg) - 1)
+    assert P % 32 == 0 and P >= rc.shape[1]
+    codes = torch.full((cols, P), 0x5A, dtype=torch.uint8, device=dev)
+    scales = torch.full((cols * P // 32,), 0x5A, dtype=torch.uint8, device=dev)
+    lib.mxfp8_quantize_sr(dev_bf16(bits, dev), codes, scales, axis=1, seed=7, offset=1,
+                          rounding=rounding, layout=layout, seg_off=torch.tensor(seg, device=dev))
+    sync()
+    used = rc.shape[1]
+    gc = host_u8(codes)
+    gs = host_u8(scales)
+    gs = gs.reshape(cols, P // 32) if layout == 0 else mma_to_rowmajor(gs, cols, P // 32)
+    assert np.array_equal(gc[:, :used], rc)
+    assert np.array_equal(gs[:, :used // 32], rs)
+    assert not gc[:, used:].any() and not gs[:, used // 32:].any()
+    st, code = lib.device_error()
+    assert st == 0 and code == 0
+
+
+def test_mxfp8_cols_bad_segments_are_reported(dev, lib):
+    """Decreasing offsets are caught by the kernel before any load: the output
+    is all zeros and the device error word says so."""
+    rows, cols = 64, 64
+    x = torch.ones(rows, cols, dtype=torch.bfloat16, device=dev)
+    seg = torch.tensor([0, 40, 30, 64], dtype=torch.int32, device=dev)
+    P = lib.mxfp8_seg_rows(rows, 3)
+    codes = torch.full((cols, P), 7, dtype=torch.uint8, device=dev)
+    scales = torch.full((cols * P // 32,), 7, dtype=torch.uint8, device=dev)
+    lib.mxfp8_quantize_sr(x, codes, scales, axis=1, seg_off=seg)
+    sync()
+    st, code = lib.device_error()
+    assert code == 16  # NVFP4MOE_DEVERR_SEGMENTS
+    assert st == 1  # NVFP4MOE_ERR_INVALID_ARG
+    assert not codes.any() and not scales.any()

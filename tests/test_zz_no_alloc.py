@@ -75,3 +75,51 @@ def test_noalloc_rejects_more_than_its_scratch(dev, lib):
     st = L.moe_route_permute_noalloc(P, P, T, E, k, d, 1, None, P, P, P, P, P, P, P, P, None)
     assert st == 4  # NVFP4MOE_ERR_WORKSPACE
     assert b"4194304" in L.nvfp4moe_last_error()
+
+
+def test_noalloc_given_amax_and_no_tokens(dev, lib):
+    """The two paths of the built-in scratch the first test does not reach: a
+    caller-supplied tensor amax (the scratch's amax slot is then not used; half
+    the true amax also saturates blocks), and T = 0 (only the expert offsets
+    and the padding of the token map are written). Each is compared with the
+    workspace entry point, run right after a call that left the scratch
+    dirty."""
+    T, E, k, d = 700, 48, 6, 512
+    logits = synth.logits_zipf_np(5, T, E)
+    lg = dev_f32(logits, dev)
+    xb = synth.rows_np(5, synth.TAG_X, 0, T, d, 1.0)
+    x = dev_bf16(xb, dev)
+    amax = dev_f32([np.abs(synth.bf16_bits_to_f32(xb)).max() * 0.5], dev)
+    for renorm in (1, 0):
+        ref = _outputs(dev, T, E, k, d)
+        ws = torch.empty(lib.moe_route_permute_workspace_size(T, E, k), dtype=torch.uint8,
+                         device=dev)
+        lib.moe_route_permute(lg, x, k, renorm, ref["idx"], ref["w"], ref["off"], ref["pos"],
+                              ref["tok"], ref["xq"], ref["xq_sc"], ref["x_ts"], ws, x_amax_in=amax)
+        got = _outputs(dev, T, E, k, d)
+        lib.moe_route_permute_noalloc(lg, x, k, renorm, got["idx"], got["w"], got["off"],
+                                      got["pos"], got["tok"], got["xq"], got["xq_sc"],
+                                      got["x_ts"], x_amax_in=amax)
+        sync()
+        _compare(ref, got)
+    # T = 0 right after a call with tokens
+    T0 = 0
+    e = torch.empty(0, dtype=torch.int32, device=dev)
+    ref = _outputs(dev, T0, E, k, d)
+    got = _outputs(dev, T0, E, k, d)
+    ref["off"].fill_(-5)
+    got["off"].fill_(-5)
+    lg0 = torch.empty(0, E, device=dev)
+    x0 = torch.empty(0, d, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(16, lib.moe_route_permute_workspace_size(T0, E, k)), dtype=torch.uint8,
+                     device=dev)
+    lib.moe_route_permute(lg0, x0, k, 1, e, torch.empty(0, device=dev), ref["off"], e, ref["tok"],
+                          ref["xq"], ref["xq_sc"], ref["x_ts"], ws)
+    lib.moe_route_permute_noalloc(lg0, x0, k, 1, e, torch.empty(0, device=dev), got["off"], e,
+                                  got["tok"], got["xq"], got["xq_sc"], got["x_ts"])
+    sync()
+    assert torch.equal(ref["off"], got["off"]) and not got["off"].any()
+    assert torch.equal(ref["tok"], got["tok"]) and (got["tok"] == -1).all()
+    assert torch.equal(ref["x_ts"], got["x_ts"])
+    st, code = lib.device_error()
+    assert st == 0 and code == 0
