@@ -713,6 +713,58 @@ def workload_name(args, shape):
 
 
 # ---------------------------------------------------------------------------
+# single-kernel cases for ncu: the backward operands' quantizers on the layer's
+# padded routed rows (dY [R_p x d], seed 7, offsets 0 / 1, MMA scale layout)
+# and the NVFP4 quantization of the activation x [T x d]
+CASES = {"mxfp8_sr_rows": "mxfp8_rows_kernel", "mxfp8_sr_cols": "mxfp8_cols_kernel",
+         "nvfp4_quantize_x": "nvfp4_quant_kernel"}
+
+
+def run_case(M, synth, torch, dev, L, calls, shape, case):
+    calls[0][1]()  # routing and dispatch: the padded row offsets
+    torch.cuda.synchronize()
+    d = shape.d
+    if case == "nvfp4_quantize_x":
+        x = L["x"]
+        codes = torch.empty(x.shape[0], d // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(x.shape[0], d // 16, dtype=torch.uint8, device=dev)
+        ts = torch.empty(1, device=dev)
+        amax = torch.empty(1, device=dev)
+        M.nvfp4moe_amax_bf16(x, amax)
+
+        def fn():
+            M.nvfp4_quantize(x, codes, scales, ts, amax_in=amax, layout=M.LAYOUT_MMA)
+        elems = x.numel()
+    else:
+        off = L["off"].cpu().numpy()
+        tok = L["tok"].cpu().numpy()
+        Rp = int(off[-1])
+        pad = torch.from_numpy(tok[:Rp] < 0).to(dev)
+        dchans = synth.outlier_channels(7, d, max(1, d // 1000))
+        dy = synth.grad_rows_torch(7, 0, Rp, d, dchans, dev)
+        dy[pad] = 0
+        axis = 0 if case == "mxfp8_sr_rows" else 1
+        codes = torch.empty((Rp, d) if axis == 0 else (d, Rp), dtype=torch.uint8, device=dev)
+        scales = torch.empty(Rp * d // 32, dtype=torch.uint8, device=dev)
+
+        def fn():
+            M.mxfp8_quantize_sr(dy, codes, scales, axis=axis, seed=7, offset=axis, layout=M.LAYOUT_MMA)
+        elems = Rp * d
+    fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.profiler.start()
+    a.record()
+    fn()
+    fn()
+    b.record()
+    torch.cuda.synchronize()
+    torch.cuda.profiler.stop()
+    print(json.dumps({"case": case, "kernel": CASES[case], "elements": elems,
+                      "ms_per_launch": round(a.elapsed_time(b) / 2, 4)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -723,6 +775,9 @@ def main():
     ap.add_argument("--router", choices=["uniform", "zipf"], default="uniform")
     ap.add_argument("--no-companions", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=sorted(CASES), default=None,
+                    help="run one kernel on the workload's tensor three times, the last two inside "
+                         "the profiler window, print its time and exit (an ncu capture case)")
     args = ap.parse_args()
     from precision_moe_numerics_quantize_b200 import synth
     shape = synth.SHAPES[args.workload]
@@ -751,6 +806,9 @@ def main():
 
     L = setup_layer(M, synth, torch, dev, shape, args.router)
     calls = layer_calls(M, L)
+    if args.case:
+        run_case(M, synth, torch, dev, L, calls, shape, args.case)
+        return
     for _ in range(args.warmup):
         for _, fn in calls:
             fn()

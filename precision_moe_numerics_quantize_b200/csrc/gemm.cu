@@ -15,7 +15,9 @@
 // tensor rate, one of N = 128 is limited by how fast one thread can issue it.
 //
 // A pipeline stage is 256 bytes of K (two 128-byte k-blocks, eight MMAs): the
-// MMA-issuing thread pays one barrier wait, one fence and one commit per stage.
+// MMA-issuing thread pays one barrier wait, one fence and one commit per stage,
+// and issues the eight MMAs from straight-line code (a loop over k-blocks with
+// a per-MMA branch on the format ran them about half again as slowly).
 // Every barrier operation costs a few hundred cycles while the tensor cores
 // and TMA keep shared memory busy, so each role does as few per stage as the
 // protocol allows.
@@ -24,7 +26,9 @@
 //   warp 0       TMA producer: first the X block scales of the stage (plain
 //                bulk copies of the one or two 128-row chunk rows) into this
 //                CTA, counted on its own `sf_loaded`; then this CTA's W and X
-//                halves (128-byte swizzle), counted on the first CTA's `full`.
+//                halves (128-byte swizzle), counted on the first CTA's `full`:
+//                one box per operand covers both k-blocks of the stage, so a
+//                stage is four TMA operations, not eight.
 //   warps 4..7   scale warps, one per TMEM lane quarter (SCALE_SETS sets of
 //                four can take turns by stage). Each lane reads the stage's X
 //                scale words from shared memory and the W scale words of its
@@ -269,6 +273,15 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
     }
 }
 
+__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *map, int32_t c0, int32_t c1,
+                                                 int32_t c2, uint32_t cbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(cbar)
+        : "memory");
+}
+
 // Instruction descriptors, M = 256 (two CTAs), N = n, K-major A and B, dense.
 __device__ __forceinline__ uint32_t idesc_nvf4(int n) {
     // a/b format E2M1 (1) at bits 7 and 10, N >> 3 at bit 17, scale format
@@ -416,10 +429,16 @@ __device__ __forceinline__ float swiglu_value(float g, float u, float alpha) {
     return __fmul_rn(__fdividef(gq, den), uq);
 }
 
+// REQUANT: the first GEMM of moe_expert_fwd_fused_requant, whose epilogue
+// warps also requantize h. It is its own instantiation: compiled into every
+// launch, the unused requantization code alone made the fp32-output GEMM
+// nearly twice as slow (3.98 ms against 7.6 ms for the full-size MXFP8 wgrad).
+template <bool REQUANT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmW,
                              const __grid_constant__ CUtensorMap tmX32,
-                             const __grid_constant__ CUtensorMap tmX64, const Params p) {
+                             const __grid_constant__ CUtensorMap tmX64,
+                             const __grid_constant__ CUtensorMap tmX96, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -454,7 +473,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         gtab[g] = e;
     }
     if (threadIdx.x == 0) *abort_flag = 0;
-    const bool requant = p.hq != nullptr;
+    constexpr bool requant = REQUANT;
     // groups without rows are never published: their decode scale is 1
     if (requant && blockIdx.x == 0)
         for (int g = threadIdx.x; g < G; g += NUM_THREADS)
@@ -491,8 +510,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             prefetch_tmap(&tmW);
             prefetch_tmap(&tmX32);
             prefetch_tmap(&tmX64);
+            prefetch_tmap(&tmX96);
             const uint32_t cfull = cluster_addr(full, 0);
             const uint32_t sfc = nvf4 ? 4 : 1;  // scale chunks per k-block
+            const int32_t gu_groups = (int32_t)(2 * p.f_out / 16);  // 16-row groups of W1 per expert
             int s = 0;
             uint32_t phase = 0, i = 0;
             // test hook: withhold every load (nothing is ever in flight), so
@@ -526,19 +547,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     for (int cr = 0; cr < xcr; ++cr)
                         bulk_load(ssf + cr * (SFX_CHUNKS * 512), p.x_sc + ((xa + cr) * p.x_nkc + kc0) * 512,
                                   nkb * sfc * 512u, &sf_loaded[sb]);
-                    if (rank == 0) mbar_arrive_expect_tx(&full[sb], (uint32_t)nkb * kblk_tx);
+                    // both k-blocks always: a lone last k-block brings its
+                    // neighbour (or the zero fill past the tensor) along
+                    if (rank == 0) mbar_arrive_expect_tx(&full[sb], 2u * kblk_tx);
                     const uint32_t cbar = cfull + 8u * sb;
-                    for (int j = 0; j < nkb; ++j) {
-                        const int32_t kx = (int32_t)(T.k0 + (int64_t)(kb0 + j) * 128);  // byte column
-                        uint8_t *sw = smem + OFF_W + s * W_STAGE + j * W_KBLK;
-                        uint8_t *sx = smem + OFF_X + s * X_STAGE + j * X_KBLK;
+                    {
+                        // one box per operand brings both k-blocks of the stage
+                        const int32_t kc = (int32_t)(T.k0 / 128 + kb0);  // k-block coordinate
+                        uint8_t *sw = smem + OFF_W + s * W_STAGE;
+                        uint8_t *sx = smem + OFF_X + s * X_STAGE;
                         if (swiglu)
-                            tma_load_5d_pair(sw, &tmW, kx, 0, 0, 8 * T.mt + 4 * (int32_t)rank, T.g, cbar);
+                            tma_load_5d_pair(sw, &tmW, 0, 0, 0, T.g * gu_groups + 8 * T.mt + 4 * (int32_t)rank, kc, cbar);
                         else
-                            tma_load_2d_pair(sw, &tmW, kx, (int32_t)w_row, cbar);
-                        if (hn >= 64) tma_load_2d_pair(sx, &tmX64, kx, xr, cbar);
-                        if (hn != 64)
-                            tma_load_2d_pair(sx + (hn >= 64 ? 8192 : 0), &tmX32, kx, xr + (hn >= 64 ? 64 : 0), cbar);
+                            tma_load_3d_pair(sw, &tmW, 0, (int32_t)w_row, kc, cbar);
+                        const CUtensorMap *mx = hn == 96 ? &tmX96 : (hn == 64 ? &tmX64 : &tmX32);
+                        tma_load_3d_pair(sx, mx, 0, xr, kc, cbar);
                     }
                     ++i;
                     if (++s == STAGES) { s = 0; phase ^= 1u; }
@@ -719,17 +742,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     const uint64_t wd = wdesc0 + (uint64_t)((s * W_STAGE) >> 4);
                     const uint64_t xd = xdesc0 + (uint64_t)((s * X_STAGE) >> 4);
                     const uint32_t sf = tmem_base + TMEM_SF + s * SF_SLOT_COLS;
-                    for (int j = 0; j < nkb; ++j) {
-                        const uint32_t sfj = sf + j * SF_KB_COLS;
+                    const uint32_t acc0 = kb0 != 0;
+                    if (nvf4) {
+                        tc_mma_nvf4_pair(tmem_base, wd, xd, idesc4, sf + 32, sf, acc0);
+                        tc_mma_nvf4_pair(tmem_base, wd + 2, xd + 2, idesc4, sf + 36, sf + 8, 1u);
+                        tc_mma_nvf4_pair(tmem_base, wd + 4, xd + 4, idesc4, sf + 40, sf + 16, 1u);
+                        tc_mma_nvf4_pair(tmem_base, wd + 6, xd + 6, idesc4, sf + 44, sf + 24, 1u);
+                        if (nkb == 2) {
+                            const uint64_t w1 = wd + (uint64_t)(W_KBLK >> 4), x1 = xd + (uint64_t)(T.n * 4);
+                            const uint32_t s1 = sf + SF_KB_COLS;
+                            tc_mma_nvf4_pair(tmem_base, w1, x1, idesc4, s1 + 32, s1, 1u);
+                            tc_mma_nvf4_pair(tmem_base, w1 + 2, x1 + 2, idesc4, s1 + 36, s1 + 8, 1u);
+                            tc_mma_nvf4_pair(tmem_base, w1 + 4, x1 + 4, idesc4, s1 + 40, s1 + 16, 1u);
+                            tc_mma_nvf4_pair(tmem_base, w1 + 6, x1 + 6, idesc4, s1 + 44, s1 + 24, 1u);
+                        }
+                    } else {
+                        for (int j = 0; j < nkb; ++j) {
+                            const uint32_t sfj = sf + j * SF_KB_COLS;
 #pragma unroll
-                        for (int kb = 0; kb < 4; ++kb) {
-                            const uint64_t woff = (uint64_t)((j * W_KBLK + 32 * kb) >> 4);
-                            const uint64_t xoff = (uint64_t)((j * X_KBLK + 32 * kb) >> 4);
-                            const uint32_t acc = (kb0 | j | kb) != 0;
-                            if (nvf4) {
-                                tc_mma_nvf4_pair(tmem_base, wd + woff, xd + xoff, idesc4, sfj + 32 + 4 * kb,
-                                                 sfj + 8 * kb, acc);
-                            } else {
+                            for (int kb = 0; kb < 4; ++kb) {
+                                const uint64_t woff = (uint64_t)((j * W_KBLK + 32 * kb) >> 4);
+                                const uint64_t xoff = (uint64_t)((j * (T.n / 2) * 128 + 32 * kb) >> 4);
+                                const uint32_t acc = (kb0 | j | kb) != 0;
                                 const uint32_t sub = (uint32_t)kb << 30;  // byte kb of the scale word
                                 tc_mma_mxf8_pair(tmem_base, wd + woff, xd + xoff, idesc_mxf8(T.n, (uint32_t)kb),
                                                  (sfj + 32) | sub, sfj | sub, acc);
@@ -897,32 +931,33 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// A [rows x cols_bytes] uint8 matrix read in boxes of 128 bytes x box_rows
-// rows with 128-byte swizzle.
-bool make_map_2d(CUtensorMap *m, const void *base, int64_t rows, int64_t cols_bytes,
-                 uint32_t box_rows) {
+// A [rows x cols_bytes] uint8 matrix seen as 3-D (128 bytes, rows, 128-byte
+// k-block): one box of (128, box_rows, 2) brings two k-blocks, each a
+// contiguous [box_rows x 128] block with 128-byte swizzle.
+bool make_map_3d_kb(CUtensorMap *m, const void *base, int64_t rows, int64_t cols_bytes,
+                    uint32_t box_rows) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)cols_bytes, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols_bytes};
-    cuuint32_t box[2] = {128, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+    cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)(cols_bytes / 128)};
+    cuuint64_t strides[2] = {(cuuint64_t)cols_bytes, 128};
+    cuuint32_t box[3] = {128, box_rows, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The [E x 2f x cols_bytes] gate/up weights seen as 5-D (bytes, 16 rows,
-// gate|up, 16-row group of h columns, expert), so that one box of
-// (128, 16, 2, 4, 1) brings 4 x (16 gate rows, the 16 matching up rows): 128
-// rows in the order the SwiGLU epilogue pairs them.
-bool make_map_swiglu(CUtensorMap *m, const void *base, int64_t E, int64_t f, int64_t cols_bytes) {
+// The [E x 2f x cols_bytes] gate/up weights seen as 5-D (128 bytes, 16 rows,
+// gate|up, 16-row group counted across experts, 128-byte k-block): one box of
+// (128, 16, 2, 4, 2) brings, for two k-blocks, 4 x (16 gate rows, the 16
+// matching up rows) = 128 rows in the order the SwiGLU epilogue pairs them.
+bool make_map_swiglu_kb(CUtensorMap *m, const void *base, int64_t E, int64_t f, int64_t cols_bytes) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     const cuuint64_t rb = (cuuint64_t)cols_bytes;
-    cuuint64_t dims[5] = {rb, 16, 2, (cuuint64_t)(f / 16), (cuuint64_t)E};
-    cuuint64_t strides[4] = {rb, (cuuint64_t)f * rb, 16 * rb, 2 * (cuuint64_t)f * rb};
-    cuuint32_t box[5] = {128, 16, 2, 4, 1};
+    cuuint64_t dims[5] = {128, 16, 2, (cuuint64_t)(E * 2 * f / 16), rb / 128};
+    cuuint64_t strides[4] = {rb, (cuuint64_t)f * rb, 16 * rb, 128};
+    cuuint32_t box[5] = {128, 16, 2, 4, 2};
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -944,16 +979,18 @@ cudaError_t launch_setup(int &grid) {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (grids[dev] == 0) {
-        e = cudaFuncSetAttribute(grouped_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_ALLOC);
-        if (e != cudaSuccess) return e;
-        // setmaxnreg only redistributes the registers the block launched
-        // with: a build that gave the kernel fewer than REGS_LAUNCH would
-        // leave the epilogue's increase waiting forever
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, grouped_gemm_pair_kernel);
-        if (e != cudaSuccess) return e;
-        if (fa.numRegs < (int)REGS_LAUNCH) return cudaErrorInvalidConfiguration;
+        for (const void *k : {reinterpret_cast<const void *>(grouped_gemm_pair_kernel<false>),
+                              reinterpret_cast<const void *>(grouped_gemm_pair_kernel<true>)}) {
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+            if (e != cudaSuccess) return e;
+            // setmaxnreg only redistributes the registers the block launched
+            // with: a build that gave the kernel fewer than REGS_LAUNCH would
+            // leave the epilogue's increase waiting forever
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, k);
+            if (e != cudaSuccess) return e;
+            if (fa.numRegs < (int)REGS_LAUNCH) return cudaErrorInvalidConfiguration;
+        }
         int sms = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (sms <= 1) sms = 148;
@@ -962,7 +999,7 @@ cudaError_t launch_setup(int &grid) {
         cfg.blockDim = dim3(NUM_THREADS);
         cfg.dynamicSmemBytes = SMEM_ALLOC;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel, &cfg) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<false>, &cfg) != cudaSuccess ||
             clusters <= 0) {
             cudaGetLastError();
             clusters = sms / 2;
@@ -1034,16 +1071,19 @@ cudaError_t launch_grouped_gemm(const GemmArgs &a, cudaStream_t s) {
     p.kt_total = (int32_t)(kbytes / 128);
     const int64_t w_rows =
         (a.group_axis == NVFP4MOE_GROUP_M) ? (int64_t)a.G * a.b_rows_per_group : a.N;
-    CUtensorMap mw, mx32, mx64;
-    const bool okw = swiglu ? make_map_swiglu(&mw, a.b, a.G, p.f_out, kbytes)
-                            : make_map_2d(&mw, a.b, w_rows, kbytes, 128);
-    if (!okw || !make_map_2d(&mx32, a.a, a.a_rows, kbytes, 32) ||
-        !make_map_2d(&mx64, a.a, a.a_rows, kbytes, 64))
+    CUtensorMap mw, mx32, mx64, mx96;
+    const bool okw = swiglu ? make_map_swiglu_kb(&mw, a.b, a.G, p.f_out, kbytes)
+                            : make_map_3d_kb(&mw, a.b, w_rows, kbytes, 128);
+    if (!okw || !make_map_3d_kb(&mx32, a.a, a.a_rows, kbytes, 32) ||
+        !make_map_3d_kb(&mx64, a.a, a.a_rows, kbytes, 64) || !make_map_3d_kb(&mx96, a.a, a.a_rows, kbytes, 96))
         return cudaErrorInvalidValue;
     int grid = 0;
     cudaError_t e = launch_setup(grid);
     if (e != cudaSuccess) return e;
-    grouped_gemm_pair_kernel<<<grid, NUM_THREADS, SMEM_ALLOC, s>>>(mw, mx32, mx64, p);
+    if (p.hq)
+        grouped_gemm_pair_kernel<true><<<grid, NUM_THREADS, SMEM_ALLOC, s>>>(mw, mx32, mx64, mx96, p);
+    else
+        grouped_gemm_pair_kernel<false><<<grid, NUM_THREADS, SMEM_ALLOC, s>>>(mw, mx32, mx64, mx96, p);
     return cudaGetLastError();
 }
 
