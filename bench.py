@@ -36,11 +36,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 expert-FFN fwd TFLOPS (% of B200 FP4 peak); quantizer HBM GB/s"
-# dram__bytes_read.sum + dram__bytes_write.sum of moe_expert_fwd's kernels per
-# call of the full-size layer: an ncu capture of the mid-size layer (one
-# kernel, a few launches), scaled to the full size by routed rows; the summary
-# is under profiles/. None while the kernels differ from the captured ones.
-EXPERT_FWD_DRAM_BYTES = None
+# dram__bytes_read.sum + dram__bytes_write.sum of moe_expert_fwd's three
+# launches (GEMM1 + SwiGLU, the grouped requantization, GEMM2) in one call of
+# the full-size layer, captured with ncu at full size (a 1-pass metric pair;
+# the summary is under profiles/). Set back to None whenever those kernels
+# change, until they are captured again.
+EXPERT_FWD_DRAM_BYTES = 10291291392
 
 
 def expert_fwd_bytes(d, f, E, rows_padded):
