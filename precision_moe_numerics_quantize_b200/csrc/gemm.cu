@@ -28,7 +28,7 @@
 //                CTA, counted on its own `sf_loaded`; then this CTA's W and X
 //                halves (128-byte swizzle), counted on the first CTA's `full`:
 //                one box per operand covers both k-blocks of the stage, so a
-//                stage is four TMA operations, not eight.
+//                stage is two tensor loads per CTA, not four.
 //   warps 4..7   scale warps, one per TMEM lane quarter (SCALE_SETS sets of
 //                four can take turns by stage). Each lane reads the stage's X
 //                scale words from shared memory and the W scale words of its
