@@ -29,8 +29,8 @@
 //                halves (128-byte swizzle), counted on the first CTA's `full`:
 //                one box per operand covers both k-blocks of the stage, so a
 //                stage is two tensor loads per CTA, not four.
-//   warps 4..7   scale warps, one per TMEM lane quarter (SCALE_SETS sets of
-//                four can take turns by stage). Each lane reads the stage's X
+//   warps 4..7   scale warps, one per TMEM lane quarter, one set for every
+//                stage (the barriers assume one set). Each lane reads the stage's X
 //                scale words from shared memory and the W scale words of its
 //                own TMEM lane, loaded from L2 one stage ahead, and writes them
 //                with tcgen05.st into the stage's scale slot in this CTA's
